@@ -1,0 +1,185 @@
+// Device helpers shared by the libsba kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sba.h"
+
+namespace sba {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxGroup = 16;
+constexpr int kMaxBlocksPerSeq = 32768;  // selection keys live in shared memory
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bounded waits give up after ~2 s
+
+// ---------------------------------------------------------------------------
+// Small arithmetic helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Order-preserving map fp32 -> u32 (larger float, larger key).  -0 is first
+// turned into +0 so that the two compare equal.
+__device__ __forceinline__ uint32_t orderable_key(float f) {
+    f = f + 0.0f;
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ void report(int32_t* status, int bit) {
+    if (status) atomicOr(status, bit);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Physical page of logical block j of sequence s, or -1 (and a status bit)
+// when the table entry is out of range.
+__device__ __forceinline__ int64_t page_of(const sba_cache& c, int s, int j, int32_t* status) {
+    int64_t p = c.block_table ? (int64_t)__ldg(c.block_table + (int64_t)s * c.max_blocks + j)
+                              : (int64_t)s * c.max_blocks + j;
+    if (p < 0 || p >= c.num_pages) {
+        report(status, SBA_DEV_BAD_PAGE);
+        return -1;
+    }
+    return p;
+}
+
+__device__ __forceinline__ int blocks_of(int len, int b) { return len <= 0 ? 0 : (len + b - 1) / b; }
+
+// Selection size for a sequence of N blocks (the rule documented in sba.h).
+__host__ __device__ __forceinline__ int num_selected(int N, const sba_select_params& p) {
+    if (N <= 0) return 0;
+    int budget = p.n_budget;
+    if (p.keep_den > 0) budget = (int)(((int64_t)N * p.keep_num + p.keep_den - 1) / p.keep_den);
+    int L = p.n_local;
+    if (p.scorer == SBA_SCORER_GATE && L < 1) L = 1;
+    if (L > N) L = N;
+    int n = budget;
+    if (p.n_min > n) n = p.n_min;
+    if (L > n) n = L;
+    return n < N ? n : N;
+}
+
+__host__ __device__ __forceinline__ int num_local(int N, const sba_select_params& p) {
+    int L = p.n_local;
+    if (p.scorer == SBA_SCORER_GATE && L < 1) L = 1;
+    return L < N ? L : (N > 0 ? N : 0);
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch (PDL): wait for the grids this one depends on;
+// let the next grid in the stream get scheduled.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// mbarrier + TMA (cp.async.bulk.tensor) wrappers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and reports
+// SBA_DEV_TIMEOUT) if the phase did not complete within kWaitTimeoutNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            report(status, SBA_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// 2-D tiled TMA load of one box into shared memory, completing on `bar`.
+// x is the innermost (element) coordinate, y the row coordinate.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level tensor-core helpers (bf16 inputs, fp32 accumulate)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D(16x8 fp32) += A(16x16 bf16, row) * B(16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+}  // namespace sba

@@ -1,0 +1,69 @@
+// Kernel launch helper: every libsba kernel is launched with programmatic
+// dependent launch enabled, so that it is scheduled while the previous kernel
+// in the stream drains; each kernel calls griddepcontrol.wait before it reads
+// anything a previous kernel may write.  SBA_PDL=0 in the environment turns
+// the attribute off (plain stream order).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdlib.h>
+
+#include "../../include/sba.h"
+
+namespace sba {
+
+inline bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("SBA_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (not a stream
+// operation, so it is also safe while a stream is being captured).
+template <auto Kernel>
+int allow_smem(int bytes) {
+    static bool done[64] = {};  // one flag set per kernel instantiation
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SBA_ERR_CUDA;
+    if (done[dev]) return SBA_OK;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return SBA_ERR_CUDA;
+    done[dev] = true;
+    return SBA_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args&&... args) {
+    if (grid.x == 0 || grid.y == 0 || grid.z == 0) return SBA_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    return e == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+}
+
+// Host-side entry points of the kernel files (validated arguments only).
+int launch_append_kv(const sba_cache& c, const void* k_new, const void* v_new, const int32_t* pos_start, int n_new,
+                     cudaStream_t stream);
+int launch_update_descriptors(const sba_cache& c, const int32_t* pos_start, int n_new, const sba_gate* gate,
+                              cudaStream_t stream);
+int score_chunk_blocks(const sba_cache& c);
+size_t score_workspace_bytes(const sba_cache& c, const sba_select_params& p);
+int launch_score_select(const sba_cache& c, const void* q, const sba_select_params& p, int32_t* sel_idx,
+                        int32_t* sel_cnt, float* gate_bias, int n_max, void* ws, cudaStream_t stream);
+int launch_sparse_decode(const sba_cache& c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
+                         const float* gate_bias, int n_max, float scale, int num_splits, float* o_part,
+                         float* lse_part, cudaStream_t stream);
+int launch_combine(const float* o_part, const float* lse_part, int B, int H_q, int S, void* out, int out_dtype,
+                   float* lse_out, cudaStream_t stream);
+
+}  // namespace sba

@@ -1,0 +1,459 @@
+// Group block scoring and shared top-n selection.
+//
+// "Rectified Sparse Attention for Efficient Long-Sequence Generation",
+// Summary: Quest-style min/max descriptors score the blocks and all query
+// heads of a GQA group share one selection; Key points: top-n that always
+// keeps the recent local blocks and a minimum count.
+// "SAS: Simple Attention Sparsification ...", Method: gate scores are
+// softmax-normalised over the historical blocks; the current block B0 keeps a
+// unit gate; the log-gates of the selected blocks go into the attention logits.
+//
+// One launch per call.  CTAs of grid (chunk, kv head, sequence) score CHUNK
+// blocks each and write fp32 scores to the workspace; the last CTA to finish a
+// (sequence, group) -- detected with a plain atomic counter, never a wait --
+// runs the selection over that group's N scores in shared memory and resets
+// the counter to zero for the next call.
+//
+// Quest score of block j for group g is
+//   sum_{qh in g} sum_c max(q_qh,c mn_c, q_qh,c mx_c) = sum_c (P_c mx_c + M_c mn_c)
+// with P_c = sum_qh max(q_qh,c, 0), M_c = sum_qh min(q_qh,c, 0): the sum over
+// the group's heads is taken once per call (reassociation only), so each block
+// costs one 256-term dot product whatever the group size.
+#include <math.h>
+
+#include "common.cuh"
+#include "launch.cuh"
+
+namespace sba {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBlocksPerWarpIter = 8;  // 4 lanes per block descriptor (512 B)
+constexpr int kRefSMs = 148;
+
+struct ScoreArgs {
+    sba_cache c;
+    const __nv_bfloat16* q;
+    sba_select_params p;
+    int32_t* sel_idx;
+    int32_t* sel_cnt;
+    float* gate_bias;
+    int n_max;
+    uint32_t* counters;  // [B][H_kv]
+    float* scores;       // Quest: [B][H_kv][mb] group scores; gate: [B][H_q][mb] logits u
+    float* mz;           // gate: [B][H_q][n_chunks][2] (chunk max, chunk sum of exp(u - max))
+    int chunk;           // blocks per CTA, multiple of 64
+};
+
+struct WsLayout {
+    size_t counters, scores, mz, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const sba_cache& c, const sba_select_params& p, int chunk) {
+    WsLayout w{};
+    const int n_chunks = (c.max_blocks + chunk - 1) / chunk;
+    size_t off = 0;
+    w.counters = off;
+    off += align256(sizeof(uint32_t) * c.B * c.H_kv);
+    w.scores = off;
+    const int rows = p.scorer == SBA_SCORER_GATE ? c.H_q : c.H_kv;
+    off += align256(sizeof(float) * (size_t)c.B * rows * c.max_blocks);
+    w.mz = off;
+    if (p.scorer == SBA_SCORER_GATE) off += align256(sizeof(float) * 2 * (size_t)c.B * c.H_q * n_chunks);
+    w.total = off;
+    return w;
+}
+
+// Exclusive prefix over the 8 warps of per-warp totals held in smem.
+__device__ __forceinline__ int warp_prefix(const int* warp_tot, int warp) {
+    int acc = 0;
+    for (int w = 0; w < warp; ++w) acc += warp_tot[w];
+    return acc;
+}
+
+// ---------------------------------------------------------------------------
+// Selection over NC ranked candidates (keys in smem) plus the forced local
+// blocks [NC, N).  Writes ascending indices to out[0..min(n_sel, n_max)).
+// k = number of candidates to take.  Runs on all 256 threads.
+// ---------------------------------------------------------------------------
+__device__ void select_and_compact(const uint32_t* keys, int NC, int N, int k, int32_t* out, int n_max,
+                                   uint32_t* hist, int* warp_tot, uint32_t* sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // mode: 0 = threshold (0 < k < NC), 1 = take all candidates, 2 = take none
+    const int mode = k >= NC ? 1 : (k <= 0 ? 2 : 0);
+    uint32_t T = 0;
+    int rem = 0;
+    if (mode == 0) {
+        uint32_t prefix = 0, pmask = 0;
+        rem = k;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            hist[tid] = 0;
+            __syncthreads();
+            for (int j = tid; j < NC; j += kThreads) {
+                const uint32_t kk = keys[j];
+                if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                uint32_t cnt[8], lsum = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    cnt[e] = hist[255 - 8 * lane - e];
+                    lsum += cnt[e];
+                }
+                uint32_t incl = lsum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const uint32_t excl = incl - lsum;
+                if (excl < (uint32_t)rem && (uint32_t)rem <= incl) {
+                    uint32_t run = excl;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (run + cnt[e] >= (uint32_t)rem) {
+                            sh[0] = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
+                            sh[1] = (uint32_t)rem - run;
+                            break;
+                        }
+                        run += cnt[e];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix = sh[0];
+            rem = (int)sh[1];
+            pmask |= 0xffu << shift;
+        }
+        T = prefix;  // exact key of the n-th candidate; `rem` equal keys are taken, lowest index first
+    }
+    // Per-warp contiguous segments, processed 32 consecutive indices at a time,
+    // so that ranks among equal keys and output positions follow index order.
+    const int seg = ((N + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+    const int jb = warp * seg, je = min(N, jb + seg);
+    const unsigned lt = (1u << lane) - 1u;
+    // pass A: ties per warp
+    int eq_w = 0;
+    if (mode == 0)
+        for (int base = jb; base < je; base += 32) {
+            const int j = base + lane;
+            const bool is_eq = j < je && j < NC && keys[j] == T;
+            eq_w += __popc(__ballot_sync(0xffffffffu, is_eq));
+        }
+    if (lane == 0) warp_tot[warp] = eq_w;
+    __syncthreads();
+    const int eq_before = warp_prefix(warp_tot, warp);
+    __syncthreads();
+    // pass B: selected per warp; pass C: write
+    for (int pass = 0; pass < 2; ++pass) {
+        int er = eq_before, sel_run = 0;
+        int out_base = 0;
+        if (pass == 1) out_base = warp_prefix(warp_tot, warp);
+        for (int base = jb; base < je; base += 32) {
+            const int j = base + lane;
+            bool sel = false, is_eq = false;
+            if (j < je) {
+                if (j >= NC) {
+                    sel = true;
+                } else if (mode == 1) {
+                    sel = true;
+                } else if (mode == 0) {
+                    const uint32_t kk = keys[j];
+                    is_eq = kk == T;
+                    sel = kk > T;
+                }
+            }
+            const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+            if (is_eq) sel = (er + __popc(eqm & lt)) < rem;
+            er += __popc(eqm);
+            const unsigned sm = __ballot_sync(0xffffffffu, sel);
+            if (pass == 1 && sel) {
+                const int pos = out_base + sel_run + __popc(sm & lt);
+                if (pos < n_max) out[pos] = j;
+            }
+            sel_run += __popc(sm);
+        }
+        if (pass == 0) {
+            __syncthreads();
+            if (lane == 0) warp_tot[warp] = sel_run;
+            __syncthreads();
+        }
+    }
+}
+
+template <int kScorer>
+__global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
+    extern __shared__ __align__(16) uint8_t dyn[];
+    __shared__ uint32_t hist[256];
+    __shared__ int warp_tot[kWarps];
+    __shared__ uint32_t sh[2];
+    __shared__ int is_last;
+    __shared__ float lse_s[kMaxGroup];
+    __shared__ __align__(16) float q_s[kMaxGroup][kHeadDim];
+
+    pdl_wait();
+    pdl_trigger();
+
+    const sba_cache& c = a.c;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int s = blockIdx.z, h = blockIdx.y, chunk_id = blockIdx.x;
+    const int G = c.H_q / c.H_kv;
+    const int mb = c.max_blocks;
+    int len = __ldg(c.seq_lens + s);
+    int N = blocks_of(len, c.b);
+    if (N > mb) {
+        if (tid == 0 && chunk_id == 0 && h == 0) report(c.status, SBA_DEV_BAD_POSITION);
+        N = mb;
+    }
+    const int L = num_local(N, a.p);
+    // blocks scored: Quest ranks [0, N-L); the gate needs u over all historical blocks [0, N-1)
+    const int n_scored = kScorer == SBA_SCORER_GATE ? max(N - 1, 0) : N - L;
+    const int j0 = chunk_id * a.chunk;
+    const int j1 = min(j0 + a.chunk, n_scored);
+
+    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn);                  // [mb] (selection)
+    float* u_s = reinterpret_cast<float*>(dyn);                          // [G][chunk] (gate, aliases keys)
+    const size_t main_words = max((size_t)mb, (size_t)G * a.chunk);
+    int* pages_s = reinterpret_cast<int*>(dyn + main_words * 4);         // [chunk]
+
+    // ---- prefetch the chunk's physical pages ----
+    for (int j = j0 + tid; j < j1; j += kThreads) {
+        const int64_t p = page_of(c, s, j, c.status);
+        pages_s[j - j0] = (int)p;
+    }
+
+    const int qt = lane & 3, sub = lane >> 2;
+    if (kScorer == SBA_SCORER_QUEST) {
+        // coefficients of this lane's 64 descriptor values: qt 0/1 = min row
+        // channels 0-63/64-127 (weights M), qt 2/3 = max row (weights P).
+        const int ch0 = (qt & 1) * 64;
+        const bool use_max = qt >= 2;
+        float coef[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) coef[e] = 0.f;
+        for (int g = 0; g < G; ++g) {
+            const uint4* qp = reinterpret_cast<const uint4*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim + ch0);
+#pragma unroll
+            for (int k8 = 0; k8 < 8; ++k8) {
+                const uint4 w = __ldg(qp + k8);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = bf16_lo(ws[e]), x1 = bf16_hi(ws[e]);
+                    coef[8 * k8 + 2 * e] += use_max ? fmaxf(x0, 0.f) : fminf(x0, 0.f);
+                    coef[8 * k8 + 2 * e + 1] += use_max ? fmaxf(x1, 0.f) : fminf(x1, 0.f);
+                }
+            }
+        }
+        __syncthreads();  // pages_s ready
+        const uint4* desc = reinterpret_cast<const uint4*>(c.desc);
+        float* out = a.scores + ((int64_t)s * c.H_kv + h) * mb;
+        for (int base = j0 + warp * kBlocksPerWarpIter; base < j1; base += kWarps * kBlocksPerWarpIter) {
+            const int j = base + sub;
+            float acc = 0.f;
+            if (j < j1) {
+                const int page = pages_s[j - j0];
+                if (page >= 0) {
+                    const uint4* ptr = desc + ((int64_t)page * c.H_kv + h) * 32 + qt * 8;
+                    uint4 w[8];
+#pragma unroll
+                    for (int k8 = 0; k8 < 8; ++k8) w[k8] = __ldg(ptr + k8);
+#pragma unroll
+                    for (int k8 = 0; k8 < 8; ++k8) {
+                        const uint32_t ws[4] = {w[k8].x, w[k8].y, w[k8].z, w[k8].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            acc = fmaf(coef[8 * k8 + 2 * e], bf16_lo(ws[e]), acc);
+                            acc = fmaf(coef[8 * k8 + 2 * e + 1], bf16_hi(ws[e]), acc);
+                        }
+                    }
+                }
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (qt == 0 && j < j1) out[j] = acc + 0.0f;
+        }
+    } else {
+        // gate: u_qh,j = q_qh . kg_j for the group's G heads; lane quarter qt owns channels qt*32..qt*32+31
+        for (int i = tid; i < G * kHeadDim; i += kThreads) {
+            const int g = i / kHeadDim, ch = i % kHeadDim;
+            q_s[g][ch] = __bfloat162float(a.q[((int64_t)s * c.H_q + h * G + g) * kHeadDim + ch]);
+        }
+        __syncthreads();
+        const float4* kg = reinterpret_cast<const float4*>(c.kg);
+        for (int base = j0 + warp * kBlocksPerWarpIter; base < j1; base += kWarps * kBlocksPerWarpIter) {
+            const int j = base + sub;
+            float acc[kMaxGroup];
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; ++g) acc[g] = 0.f;
+            if (j < j1) {
+                const int page = pages_s[j - j0];
+                if (page >= 0) {
+                    const float4* ptr = kg + ((int64_t)page * c.H_kv + h) * 32 + qt * 8;
+                    float4 w[8];
+#pragma unroll
+                    for (int k8 = 0; k8 < 8; ++k8) w[k8] = __ldg(ptr + k8);
+#pragma unroll
+                    for (int k8 = 0; k8 < 8; ++k8) {
+#pragma unroll
+                        for (int g = 0; g < kMaxGroup; ++g) {
+                            if (g < G) {
+                                const float4 qv = *reinterpret_cast<const float4*>(&q_s[g][qt * 32 + 4 * k8]);
+                                acc[g] = fmaf(qv.x, w[k8].x, acc[g]);
+                                acc[g] = fmaf(qv.y, w[k8].y, acc[g]);
+                                acc[g] = fmaf(qv.z, w[k8].z, acc[g]);
+                                acc[g] = fmaf(qv.w, w[k8].w, acc[g]);
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; ++g) {
+                if (g < G) {
+                    float v = acc[g];
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    if (qt == 0 && j < j1) {
+                        a.scores[((int64_t)s * c.H_q + h * G + g) * mb + j] = v;
+                        u_s[g * a.chunk + (j - j0)] = v;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        // per-head (max, sum exp(u - max)) of this chunk
+        const int n_chunks = gridDim.x;
+        for (int g = warp; g < G; g += kWarps) {
+            float m = -INFINITY;
+            for (int i = lane; i < j1 - j0; i += 32) m = fmaxf(m, u_s[g * a.chunk + i]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float z = 0.f;
+            if (m > -INFINITY)
+                for (int i = lane; i < j1 - j0; i += 32) z += expf(u_s[g * a.chunk + i] - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            if (lane == 0) {
+                float* dst = a.mz + (((int64_t)s * c.H_q + h * G + g) * n_chunks + chunk_id) * 2;
+                dst[0] = m;
+                dst[1] = z;
+            }
+        }
+    }
+
+    // ---- completion count: the last CTA of this (sequence, group) selects ----
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t prev = atomicAdd(a.counters + s * c.H_kv + h, 1u);
+        is_last = prev == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+
+    const int n_sel = num_selected(N, a.p);
+    const int NC = N - L;  // ranked candidates [0, NC); locals [NC, N)
+    const int k = n_sel - L;
+    if (kScorer == SBA_SCORER_QUEST) {
+        const float* sc = a.scores + ((int64_t)s * c.H_kv + h) * mb;
+        for (int j = tid; j < NC; j += kThreads) keys[j] = orderable_key(__ldcg(sc + j));
+    } else {
+        const int n_chunks = gridDim.x;
+        for (int g = warp; g < G; g += kWarps) {
+            const float* mzp = a.mz + ((int64_t)s * c.H_q + h * G + g) * n_chunks * 2;
+            float M = -INFINITY;
+            for (int i = lane; i < n_chunks; i += 32) M = fmaxf(M, __ldcg(mzp + 2 * i));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            float Z = 0.f;
+            if (M > -INFINITY)
+                for (int i = lane; i < n_chunks; i += 32) {
+                    const float m = __ldcg(mzp + 2 * i);
+                    if (m > -INFINITY) Z += __ldcg(mzp + 2 * i + 1) * expf(m - M);
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+            if (lane == 0) lse_s[g] = M > -INFINITY ? M + logf(Z) : -INFINITY;
+        }
+        __syncthreads();
+        for (int j = tid; j < NC; j += kThreads) {
+            float sc = 0.f;
+            for (int g = 0; g < G; ++g)
+                sc += expf(__ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j) - lse_s[g]);
+            keys[j] = orderable_key(sc);
+        }
+    }
+    __syncthreads();
+    int32_t* out = a.sel_idx + ((int64_t)s * c.H_kv + h) * a.n_max;
+    select_and_compact(keys, NC, N, k, out, a.n_max, hist, warp_tot, sh);
+    if (n_sel > a.n_max && tid == 0) report(c.status, SBA_DEV_BAD_SELECTION);
+    const int n_out = min(n_sel, a.n_max);
+    if (tid == 0) a.sel_cnt[s * c.H_kv + h] = n_out;
+    if (kScorer == SBA_SCORER_GATE && a.gate_bias != nullptr) {
+        __syncthreads();
+        for (int i = tid; i < n_out * G; i += kThreads) {
+            const int pos = i / G, g = i % G;
+            const int j = __ldcg(out + pos);
+            const float bias =
+                j == N - 1 ? 0.f : __ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j) - lse_s[g];
+            a.gate_bias[((int64_t)s * c.H_q + h * G + g) * a.n_max + pos] = bias;
+        }
+    }
+    if (tid == 0) a.counters[s * c.H_kv + h] = 0u;  // ready for the next call
+}
+
+}  // namespace
+
+int score_chunk_blocks(const sba_cache& c) {
+    int chunk = kWarps * kBlocksPerWarpIter;
+    const int64_t units = (int64_t)c.B * c.H_kv;
+    while (chunk < 1024 && units * ((c.max_blocks + chunk - 1) / chunk) > 4 * kRefSMs) chunk *= 2;
+    return chunk;
+}
+
+size_t score_workspace_bytes(const sba_cache& c, const sba_select_params& p) {
+    return ws_layout(c, p, score_chunk_blocks(c)).total;
+}
+
+static size_t score_smem_bytes(const sba_cache& c, int chunk) {
+    const int G = c.H_q / c.H_kv;
+    const size_t main_words = c.max_blocks > G * chunk ? (size_t)c.max_blocks : (size_t)G * chunk;
+    return main_words * 4 + (size_t)chunk * 4;
+}
+
+int launch_score_select(const sba_cache& c, const void* q, const sba_select_params& p, int32_t* sel_idx,
+                        int32_t* sel_cnt, float* gate_bias, int n_max, void* ws, cudaStream_t stream) {
+    const int chunk = score_chunk_blocks(c);
+    const WsLayout w = ws_layout(c, p, chunk);
+    ScoreArgs a{};
+    a.c = c;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.p = p;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.gate_bias = gate_bias;
+    a.n_max = n_max;
+    a.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + w.counters);
+    a.scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.scores);
+    a.mz = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.mz);
+    a.chunk = chunk;
+    const size_t smem = score_smem_bytes(c, chunk);
+    dim3 grid((c.max_blocks + chunk - 1) / chunk, c.H_kv, c.B);
+    constexpr int kMaxSmem = 227 * 1024;
+    if (smem > (size_t)kMaxSmem) return SBA_ERR_UNSUPPORTED;
+    if (p.scorer == SBA_SCORER_GATE) {
+        if (allow_smem<score_select_kernel<SBA_SCORER_GATE>>(kMaxSmem) != SBA_OK) return SBA_ERR_CUDA;
+        return launch(score_select_kernel<SBA_SCORER_GATE>, grid, dim3(kThreads), smem, stream, a);
+    }
+    if (allow_smem<score_select_kernel<SBA_SCORER_QUEST>>(kMaxSmem) != SBA_OK) return SBA_ERR_CUDA;
+    return launch(score_select_kernel<SBA_SCORER_QUEST>, grid, dim3(kThreads), smem, stream, a);
+}
+
+}  // namespace sba

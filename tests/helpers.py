@@ -41,3 +41,83 @@ def gather_tokens(c: O.Cache, s: int, h: int, which: str = "k") -> np.ndarray:
         p = int(c.block_table[s, j]) if c.block_table is not None else s * c.max_blocks + j
         rows.append(bf16_to_f64(arr[p, h, t % c.b]))
     return np.array(rows).reshape(L, c.d)
+
+
+# ---------------------------------------------------------------------------
+# GPU-side helpers (used only by tests marked gpu)
+# ---------------------------------------------------------------------------
+
+ATOL_OUT = 2e-3        # attention output, max-abs (bf16 inputs, fp32 accumulation)
+NEAR_TIE_REL = 1e-5    # near-tie band for selection differences
+
+
+def gpu_cache(w: W.Workload, lay: W.Layout, li: W.LayerInputs, max_len=None):
+    """Device tensors of one layer with zeroed descriptors and a status word."""
+    from block_sparse_gqa_min_b200 import sba
+
+    dev = torch.device("cuda")
+    k, v = li.k.to(dev), li.v.to(dev)
+    c = sba.Cache(
+        k=k, v=v, seq_lens=lay.seq_lens.to(dev, torch.int32), H_q=w.H_q, max_blocks=lay.max_blocks,
+        max_len=int(max_len if max_len is not None else lay.seq_lens.max().item()),
+        block_table=None if lay.block_table is None else lay.block_table.to(dev, torch.int32),
+        desc=torch.zeros((lay.num_pages, w.H_kv, 2, w.d), dtype=torch.bfloat16, device=dev)
+        if w.scorer == "quest" else None,
+        kg=torch.zeros((lay.num_pages, w.H_kv, w.d), dtype=torch.float32, device=dev)
+        if w.scorer == "gate" else None,
+        status=torch.zeros((1,), dtype=torch.int32, device=dev),
+    )
+    return c
+
+
+def fill_descriptors(c, w: W.Workload, li: W.LayerInputs):
+    from block_sparse_gqa_min_b200 import sba
+
+    pos0 = torch.zeros((c.B,), dtype=torch.int32, device=c.k.device)
+    if w.scorer == "gate":
+        sba.sba_update_descriptors(c, pos0, c.max_len, li.Wq.cuda(), li.Wk.cuda())
+    else:
+        sba.sba_update_descriptors(c, pos0, c.max_len)
+
+
+def params_of(w: W.Workload):
+    from block_sparse_gqa_min_b200 import sba
+
+    return sba.select_params(w.n_budget, w.n_local, w.n_min, w.keep_num, w.keep_den,
+                             sba.SBA_SCORER_GATE if w.scorer == "gate" else sba.SBA_SCORER_QUEST)
+
+
+def oracle_decode(w: W.Workload, oc: O.Cache, li: W.LayerInputs, n_max=None):
+    kw = dict(scale=w.scale, n_budget=w.n_budget, n_local=w.n_local, n_min=w.n_min,
+              keep_num=w.keep_num, keep_den=w.keep_den, scorer=w.scorer, n_max=n_max)
+    if w.scorer == "gate":
+        kw.update(Wq=li.Wq.cpu().numpy(), Wk=li.Wk.cpu().numpy())
+    return O.decode(oc, W.bf16_bits(li.q), **kw)
+
+
+def check_selection(ref: O.Decoded, sel_idx: np.ndarray, sel_cnt: np.ndarray, oc: O.Cache, w: W.Workload):
+    """Bit-exact block sets, or differences confined to near-ties of the oracle's
+    own scores (|s - theta| <= 1e-5 |theta|, theta = score of the last block the
+    oracle admitted).  Returns the number of (sequence, group) near-tie events."""
+    events = 0
+    L_eff = max(w.n_local, 1) if w.scorer == "gate" else w.n_local
+    for s in range(oc.B):
+        N = int(oc.n_blocks()[s])
+        L = min(L_eff, N)
+        for h in range(oc.H_kv):
+            n_ref = int(ref.sel_cnt[s, h])
+            assert int(sel_cnt[s, h]) == n_ref, (s, h, int(sel_cnt[s, h]), n_ref)
+            a = set(ref.sel_idx[s, h, :n_ref].tolist())
+            b = sel_idx[s, h, :n_ref].tolist()
+            assert b == sorted(b), "selection must ascend"
+            if a == set(b):
+                continue
+            events += 1
+            sc = ref.score[s, h, : N - L].astype(np.float32).astype(np.float64)
+            admitted = [j for j in a if j < N - L]
+            theta = min(sc[j] for j in admitted)
+            diff = a.symmetric_difference(b)
+            for j in diff:
+                assert j < N - L, "a local block differs"
+                assert abs(sc[j] - theta) <= NEAR_TIE_REL * abs(theta), (s, h, j, sc[j], theta)
+    return events

@@ -1,0 +1,270 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Selections must match bit-exactly (near-ties of the oracle's own scores
+within 1e-5 relative are resolved by re-running the oracle on the GPU's
+selection); outputs within 2e-3 max-abs; descriptors exactly (Quest) or to
+fp32 rounding (gate)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from block_sparse_gqa_min_b200 import sba
+from block_sparse_gqa_min_b200 import workloads as W
+from tests.helpers import (ATOL_OUT, bf16_to_f64, check_selection, fill_descriptors, gpu_cache, make_case,
+                           oracle_cache, oracle_decode, params_of, small_workload)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+def run_case(w: W.Workload, seed=0, num_splits=None, layout=None, layer_inputs=None, check_desc=True,
+             device="cpu"):
+    lay = layout or W.make_layout(w, seed, device=device)
+    li = layer_inputs or W.make_layer(w, lay, seed, 0, device=device)
+    c = gpu_cache(w, lay, li)
+    fill_descriptors(c, w, li)
+    p = params_of(w)
+    bufs = sba.alloc_step(c, p, num_splits=num_splits)
+    q = li.q.cuda()
+    sba.decode_step(c, q, p, bufs, w.scale)
+    torch.cuda.synchronize()
+    oc = oracle_cache(w, lay, li)
+    ref = oracle_decode(w, oc, li, n_max=bufs.sel_idx.shape[-1])
+    sel_idx = bufs.sel_idx.cpu().numpy()
+    sel_cnt = bufs.sel_cnt.cpu().numpy()
+    events = check_selection(ref, sel_idx, sel_cnt, oc, w)
+    expect = ref
+    if events:
+        bias = ref.logg if w.scorer == "gate" else None
+        out, lse = O.attend(oc, W.bf16_bits(li.q), sel_idx, sel_cnt, w.scale, bias)
+        expect = O.Decoded(ref.score, sel_idx, sel_cnt, ref.logg, out, lse)
+    out = bufs.out.float().cpu().numpy()
+    err = np.abs(out - expect.out).max()
+    assert err <= ATOL_OUT, err
+    lse = bufs.lse.cpu().numpy()
+    fin = np.isfinite(expect.lse)
+    assert np.array_equal(np.isfinite(lse), fin)
+    assert np.abs(lse[fin] - expect.lse[fin]).max(initial=0) <= 1e-3
+    if w.scorer == "gate":
+        gb = bufs.gate_bias.cpu().numpy()
+        for s in range(w.B):
+            for qh in range(w.H_q):
+                h = qh // w.G
+                n = sel_cnt[s, h]
+                want = expect.logg[s, qh, sel_idx[s, h, :n]]
+                np.testing.assert_allclose(gb[s, qh, :n], want, rtol=0, atol=5e-5)
+    assert int(c.status.item()) == 0
+    if check_desc:
+        check_descriptors(w, lay, li, c, oc)
+    return dict(events=events, err=float(err), c=c, bufs=bufs, ref=ref, lay=lay, li=li)
+
+
+def check_descriptors(w, lay, li, c, oc):
+    """Device descriptors against the oracle's, page by page."""
+    B = w.B
+    nblk = oc.n_blocks()
+    if w.scorer == "quest":
+        mn, mx = O.quest_desc(oc)
+        d = c.desc.float().cpu().numpy()
+        for s in range(B):
+            for j in range(int(nblk[s])):
+                p = int(oc.block_table[s, j]) if oc.block_table is not None else s * oc.max_blocks + j
+                assert np.array_equal(d[p, :, 0, :], mn[s, j]), (s, j)
+                assert np.array_equal(d[p, :, 1, :], mx[s, j]), (s, j)
+    else:
+        _, kg = O.gate_desc(oc, li.Wk.cpu().numpy())
+        Wq = li.Wq.cpu().numpy().astype(np.float64)
+        dg = Wq.shape[0]
+        got = c.kg.cpu().numpy()
+        for s in range(B):
+            for j in range(int(nblk[s])):
+                p = int(oc.block_table[s, j]) if oc.block_table is not None else s * oc.max_blocks + j
+                want = kg[s, j] @ Wq / math.sqrt(dg)          # [H_kv][d]
+                np.testing.assert_allclose(got[p], want, rtol=1e-4, atol=1e-4 * np.abs(want).max())
+
+
+# ----------------------------------------------------------------------------
+# the tiny workload, exactly as specified
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_workload(seed):
+    w = W.WORKLOADS["tiny"]
+    r = run_case(w, seed)
+    sel = r["bufs"].sel_idx.cpu().numpy()[0]
+    hot = r["li"].hot
+    # hot blocks (keys aligned with the group's mean query) should be picked
+    for h in range(w.H_kv):
+        assert set(hot) <= set(sel[h].tolist())
+
+
+# ----------------------------------------------------------------------------
+# randomized shapes and edge cases
+# ----------------------------------------------------------------------------
+
+CASES = [
+    dict(H_q=8, H_kv=2, b=64, len_lo=1000, len_hi=1000, n_budget=5, n_local=2),     # ragged tail
+    dict(H_q=4, H_kv=4, b=64, len_lo=1, len_hi=1, n_budget=4, n_local=1),           # one token
+    dict(H_q=16, H_kv=1, b=64, len_lo=63, len_hi=63, n_budget=4, n_local=0),        # G 16, one partial block
+    dict(H_q=7, H_kv=1, b=128, len_lo=3001, len_hi=3001, n_budget=6, n_local=2),    # G 7, b 128
+    dict(H_q=10, H_kv=2, b=64, len_lo=700, len_hi=2100, B=3, n_budget=7, n_local=2, paged=True),
+    dict(H_q=8, H_kv=8, b=64, len_lo=640, len_hi=640, n_budget=100, n_local=2),     # n >= N: dense
+    dict(H_q=8, H_kv=2, b=64, len_lo=2000, len_hi=2000, n_budget=3, n_local=3),     # L = n
+    dict(H_q=8, H_kv=2, b=64, len_lo=4000, len_hi=4000, n_budget=2, n_local=1, n_min=9),   # min count wins
+    dict(H_q=28, H_kv=4, b=128, len_lo=20000, len_hi=20000, n_local=4, n_min=4, keep_num=5, keep_den=100),
+    dict(H_q=6, H_kv=3, b=128, len_lo=129, len_hi=4000, B=4, n_budget=5, n_local=1, paged=True),
+    dict(H_q=32, H_kv=8, b=64, len_lo=7000, len_hi=9000, B=2, n_budget=12, n_local=2, n_min=4, paged=True,
+         channel_scale_sigma=0.5),
+]
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_random_shapes(case):
+    w = small_workload(d=128, **CASES[case])
+    for seed in (0, 1):
+        run_case(w, seed)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 5, 16])
+def test_split_counts_agree(splits):
+    w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=3000, len_hi=3000, n_budget=11, n_local=2)
+    run_case(w, 3, num_splits=splits)
+
+
+def test_exact_ties_go_to_lower_index():
+    """Copies of one page give bit-identical scores on both sides; the lower
+    logical index must win."""
+    w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=64 * 20, len_hi=64 * 20, n_budget=5, n_local=1)
+    lay = W.make_layout(w, 0)
+    li = W.make_layer(w, lay, 0, 0)
+    for p in (3, 7, 9, 12, 15):
+        li.k[p] = li.k[2]
+    r = run_case(w, 0, layout=lay, layer_inputs=li)
+    assert r["events"] == 0
+
+
+def test_empty_sequence_in_batch():
+    w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=500, len_hi=500, B=3, n_budget=4, n_local=1)
+    lay = W.make_layout(w, 0)
+    lay.seq_lens[1] = 0
+    run_case(w, 0, layout=lay)
+
+
+# ----------------------------------------------------------------------------
+# gate scorer + SAS log-gate
+# ----------------------------------------------------------------------------
+
+GATE_CASES = [
+    dict(H_q=10, H_kv=2, b=64, len_lo=3000, len_hi=3000, n_budget=6, n_local=2),
+    dict(H_q=5, H_kv=1, b=64, len_lo=65, len_hi=65, n_budget=4, n_local=2),          # C = 1
+    dict(H_q=8, H_kv=4, b=128, len_lo=200, len_hi=5000, B=3, n_budget=5, n_local=0, paged=True),
+    dict(H_q=40, H_kv=8, b=64, len_lo=9000, len_hi=9000, n_budget=32, n_local=2, n_min=16),
+]
+
+
+@pytest.mark.parametrize("case", range(len(GATE_CASES)))
+def test_gate_shapes(case):
+    w = small_workload(d=128, scorer="gate", dg=128, **GATE_CASES[case])
+    for seed in (0, 1):
+        run_case(w, seed)
+
+
+# ----------------------------------------------------------------------------
+# append + descriptor maintenance
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("scorer", ["quest", "gate"])
+def test_append_then_update_matches_recompute(scorer):
+    w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=1500, len_hi=2300, B=3, n_budget=6, n_local=2,
+                       paged=True, scorer=scorer, append_tokens=40, dg=128)
+    lay = W.make_layout(w, 4)
+    li = W.make_layer(w, lay, 4, 0)
+    c = gpu_cache(w, lay, li, max_len=w.max_blocks * w.b)
+    fill_descriptors(c, w, li)
+    # overwrite the last 40 positions of every sequence (a rectification window)
+    pos = (lay.seq_lens - 40).to(torch.int32).cuda()
+    kn, vn = li.k_new.cuda(), li.v_new.cuda()
+    sba.sba_append_kv(c, kn, vn, pos)
+    if scorer == "gate":
+        sba.sba_update_descriptors(c, pos, 40, li.Wq.cuda(), li.Wk.cuda())
+    else:
+        sba.sba_update_descriptors(c, pos, 40)
+    torch.cuda.synchronize()
+    assert int(c.status.item()) == 0
+    li2 = W.LayerInputs(li.q, c.k.cpu(), c.v.cpu(), li.k_new, li.v_new, li.Wq, li.Wk)
+    # the appended rows landed where the block table says
+    oc = oracle_cache(w, lay, li2)
+    from tests.helpers import gather_tokens
+    for s in range(w.B):
+        L = int(lay.seq_lens[s])
+        for h in range(w.H_kv):
+            keys = gather_tokens(oc, s, h, "k")[L - 40:L]
+            vals = gather_tokens(oc, s, h, "v")[L - 40:L]
+            np.testing.assert_array_equal(keys, li.k_new[s, :, h].float().numpy())
+            np.testing.assert_array_equal(vals, li.v_new[s, :, h].float().numpy())
+    check_descriptors(w, lay, li2, c, oc)
+
+
+# ----------------------------------------------------------------------------
+# combine
+# ----------------------------------------------------------------------------
+
+def test_combine_against_oracle():
+    g = torch.Generator().manual_seed(0)
+    B, H, S = 3, 5, 9
+    o = torch.randn((B, H, S, 128), generator=g)
+    lse = torch.randn((B, H, S), generator=g) * 3
+    lse[0, 0, :] = -math.inf
+    lse[1, 2, ::2] = -math.inf
+    out = torch.empty((B, H, 128), device="cuda")
+    lo = torch.empty((B, H), device="cuda")
+    sba.sba_combine(o.cuda(), lse.cuda(), out, lo)
+    ob = torch.empty((B, H, 128), device="cuda", dtype=torch.bfloat16)
+    sba.sba_combine(o.cuda(), lse.cuda(), ob)
+    torch.cuda.synchronize()
+    want, wl = O.combine(o.double().numpy(), lse.double().numpy())
+    np.testing.assert_allclose(out.cpu().numpy(), want, rtol=0, atol=1e-5)
+    fin = np.isfinite(wl)
+    np.testing.assert_allclose(lo.cpu().numpy()[fin], wl[fin], rtol=0, atol=1e-5)
+    assert np.all(lo.cpu().numpy()[~fin] == -np.inf)
+    np.testing.assert_allclose(ob.float().cpu().numpy(), want, rtol=1 / 128, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# device-side error reporting (no trap, no fault)
+# ----------------------------------------------------------------------------
+
+def test_bad_block_table_entry_is_reported_not_read():
+    w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=2000, len_hi=2000, B=2, n_budget=4, n_local=1,
+                       paged=True)
+    lay = W.make_layout(w, 0)
+    li = W.make_layer(w, lay, 0, 0)
+    c = gpu_cache(w, lay, li)
+    fill_descriptors(c, w, li)
+    c.block_table[1, 5] = 10 ** 6          # outside [0, num_pages)
+    c.block_table[0, 3] = -7
+    p = params_of(w)
+    bufs = sba.alloc_step(c, p)
+    sba.decode_step(c, li.q.cuda(), p, bufs, w.scale)
+    torch.cuda.synchronize()
+    assert int(c.status.item()) & sba.SBA_DEV_BAD_PAGE
+
+
+def test_bad_selection_index_is_reported_not_read():
+    w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=1000, len_hi=1000, n_budget=4, n_local=1)
+    lay = W.make_layout(w, 0)
+    li = W.make_layer(w, lay, 0, 0)
+    c = gpu_cache(w, lay, li)
+    sel = torch.tensor([[[0, 3, 5000, 15], [1, -2, 4, 15]]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[4, 4]], dtype=torch.int32, device="cuda")
+    o = torch.empty((1, 8, 2, 128), device="cuda")
+    lse = torch.empty((1, 8, 2), device="cuda")
+    sba.sba_sparse_decode(c, li.q.cuda(), sel, cnt, None, w.scale, o, lse)
+    torch.cuda.synchronize()
+    assert int(c.status.item()) & sba.SBA_DEV_BAD_SELECTION
+    assert torch.isfinite(o).all()
