@@ -8,6 +8,14 @@
 
 using namespace sba;
 
+namespace sba {
+namespace {
+thread_local cudaError_t g_last = cudaSuccess;
+}
+void note_cuda_error(cudaError_t e) { g_last = e; }
+cudaError_t last_cuda_error() { return g_last; }
+}  // namespace sba
+
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -42,7 +50,10 @@ int check_params(const sba_select_params* p) {
 
 int after_launch(int rc) {
     if (rc != SBA_OK) return rc;
-    return cudaGetLastError() == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return SBA_OK;
+    note_cuda_error(e);
+    return SBA_ERR_CUDA;
 }
 
 }  // namespace
@@ -58,6 +69,11 @@ const char* sba_status_string(int status) {
         case SBA_ERR_CUDA: return "CUDA launch or runtime error";
         default: return "unknown status";
     }
+}
+
+const char* sba_last_cuda_error(void) {
+    const cudaError_t e = last_cuda_error();
+    return e == cudaSuccess ? "no error" : cudaGetErrorString(e);
 }
 
 int32_t sba_num_selected(int32_t N, const sba_select_params* p) {

@@ -20,17 +20,27 @@ inline bool pdl_enabled() {
     return on;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device (not a stream
-// operation, so it is also safe while a stream is being captured).
+// Record the last CUDA error of a library call (for sba_last_cuda_error).
+void note_cuda_error(cudaError_t e);
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` when the current
+// limit is lower (not a stream operation, so it is safe during capture).
 template <auto Kernel>
 int allow_smem(int bytes) {
-    static bool done[64] = {};  // one flag set per kernel instantiation
+    static int allowed[64] = {};  // per device, per kernel instantiation
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SBA_ERR_CUDA;
-    if (done[dev]) return SBA_OK;
-    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        note_cuda_error(e);
         return SBA_ERR_CUDA;
-    done[dev] = true;
+    }
+    if (bytes <= 48 * 1024 || bytes <= allowed[dev]) return SBA_OK;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return SBA_ERR_CUDA;
+    }
+    allowed[dev] = bytes;
     return SBA_OK;
 }
 
@@ -48,7 +58,11 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStr
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-    return e == cudaSuccess ? SBA_OK : SBA_ERR_CUDA;
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return SBA_ERR_CUDA;
+    }
+    return SBA_OK;
 }
 
 // Host-side entry points of the kernel files (validated arguments only).

@@ -446,13 +446,12 @@ int launch_score_select(const sba_cache& c, const void* q, const sba_select_para
     a.chunk = chunk;
     const size_t smem = score_smem_bytes(c, chunk);
     dim3 grid((c.max_blocks + chunk - 1) / chunk, c.H_kv, c.B);
-    constexpr int kMaxSmem = 227 * 1024;
-    if (smem > (size_t)kMaxSmem) return SBA_ERR_UNSUPPORTED;
+    if (smem > (size_t)200 * 1024) return SBA_ERR_UNSUPPORTED;
     if (p.scorer == SBA_SCORER_GATE) {
-        if (allow_smem<score_select_kernel<SBA_SCORER_GATE>>(kMaxSmem) != SBA_OK) return SBA_ERR_CUDA;
+        if (allow_smem<score_select_kernel<SBA_SCORER_GATE>>((int)smem) != SBA_OK) return SBA_ERR_CUDA;
         return launch(score_select_kernel<SBA_SCORER_GATE>, grid, dim3(kThreads), smem, stream, a);
     }
-    if (allow_smem<score_select_kernel<SBA_SCORER_QUEST>>(kMaxSmem) != SBA_OK) return SBA_ERR_CUDA;
+    if (allow_smem<score_select_kernel<SBA_SCORER_QUEST>>((int)smem) != SBA_OK) return SBA_ERR_CUDA;
     return launch(score_select_kernel<SBA_SCORER_QUEST>, grid, dim3(kThreads), smem, stream, a);
 }
 

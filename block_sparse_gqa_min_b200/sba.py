@@ -35,7 +35,10 @@ SBA_OUT_BF16 = 1
 
 class SbaError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {sba_status_string(code)} (status {code})")
+        msg = f"{where}: {sba_status_string(code)} (status {code})"
+        if code == SBA_ERR_CUDA:
+            msg += f": {load().sba_last_cuda_error().decode()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -78,6 +81,7 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int32
 _SIGS = {
     "sba_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "sba_last_cuda_error": ([], ctypes.c_char_p),
     "sba_num_selected": ([_I, ctypes.POINTER(sba_select_params)], _I),
     "sba_budget_from_sparsity": ([_I, _I, _I], _I),
     "sba_default_num_splits": ([ctypes.POINTER(sba_cache), _I, _I], _I),

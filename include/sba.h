@@ -137,6 +137,10 @@ typedef struct sba_select_params {
 /* Message for a status code (static string, never NULL). */
 const char *sba_status_string(int status);
 
+/* Text of the last CUDA error a call of this thread returned SBA_ERR_CUDA for
+ * ("no error" if none); static string, never NULL. */
+const char *sba_last_cuda_error(void);
+
 /* Host helper: blocks selected for a sequence of N blocks under `p` (the rule
  * above).  Returns -1 if p is NULL. */
 int32_t sba_num_selected(int32_t N, const sba_select_params *p);
