@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--path", default="fused", choices=["fused", "separate"],
+                    help="fused: one sba_decode_step launch per layer; separate: the five single-step calls")
     return ap.parse_args()
 
 
@@ -188,18 +190,27 @@ def build_layers(w, lay, seed, n_layers, dev):
         if ws is None:
             ws = bufs.ws
         bufs.ws = ws  # calls are stream-ordered, so layers share one workspace
-        layers.append(dict(c=c, li=li, bufs=bufs))
+        A = None
+        if gate:
+            A = torch.empty((w.d, 3 * w.d), dtype=torch.float32, device=dev)
+            sba.sba_fold_gate(li.Wq, li.Wk, A)
+        layers.append(dict(c=c, li=li, bufs=bufs, A=A))
     # positions of the step's re-appended tokens: the last `append_tokens` positions
     pos = (lay.seq_lens - w.append_tokens).clamp(min=0).to(torch.int32)
     torch.cuda.synchronize()
     return layers, p, pos
 
 
-def layer_step(w, L, p, pos, q=None, k_new=None, v_new=None):
+def layer_step(w, L, p, pos, q=None, k_new=None, v_new=None, path="fused"):
     from block_sparse_gqa_min_b200 import sba
 
     c, li, bufs = L["c"], L["li"], L["bufs"]
     q = li.q if q is None else q
+    if path == "fused":
+        sba.sba_decode_step(c, q, p, w.scale, bufs.out, bufs.lse, k_new=li.k_new if k_new is None else k_new,
+                            v_new=li.v_new if v_new is None else v_new, pos_start=pos, gate_A=L["A"],
+                            sel_idx=bufs.sel_idx, sel_cnt=bufs.sel_cnt, gate_bias=bufs.gate_bias)
+        return
     sba.sba_append_kv(c, li.k_new if k_new is None else k_new, li.v_new if v_new is None else v_new, pos)
     if w.scorer == "gate":
         sba.sba_update_descriptors(c, pos, w.append_tokens, li.Wq, li.Wk)
@@ -208,7 +219,7 @@ def layer_step(w, L, p, pos, q=None, k_new=None, v_new=None):
     sba.decode_step(c, q, p, bufs, w.scale)
 
 
-KERNELS_PER_LAYER = 5  # append, update, score+select, sparse decode, combine
+KERNELS_PER_LAYER = {"fused": 1, "separate": 5}  # separate: append, update, score+select, decode, combine
 
 
 def native(args, rank, world, local):
@@ -236,7 +247,7 @@ def native(args, rank, world, local):
 
     def step():
         for L in layers:
-            layer_step(w, L, p, pos)
+            layer_step(w, L, p, pos, path=args.path)
 
     # capture one step in a CUDA graph
     side = torch.cuda.Stream()
@@ -287,26 +298,47 @@ def native(args, rank, world, local):
     ms_max = max_over_ranks(total_ms / args.steps, world, dev)
     value = job_gbs(step_bytes, world, ms_max)
 
-    # ---- per-kernel durations, measured live on the launching stream ----
-    kt = {"score_select": [], "sparse_decode": [], "combine": []}
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    # ---- per-launch durations, measured live on the launching stream ----
+    # launches are queued behind a sleep kernel so that host-side gaps between
+    # them do not appear in the device-side event intervals
+    names = ["decode_step"] if args.path == "fused" else ["append_kv", "update_descriptors", "score_select",
+                                                          "sparse_decode", "combine"]
+    kt = {k: [] for k in names}
     for _ in range(3):
+        torch.cuda._sleep(int(2e8))
+        rec = []
         for L in layers:
             c, li, bufs = L["c"], L["li"], L["bufs"]
-            evs[0].record()
-            sba.sba_score_select(c, li.q, p, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, bufs.ws)
-            evs[1].record()
-            sba.sba_sparse_decode(c, li.q, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, w.scale, bufs.o_part,
-                                  bufs.lse_part)
-            evs[2].record()
-            sba.sba_combine(bufs.o_part, bufs.lse_part, bufs.out, bufs.lse)
-            evs[3].record()
-            torch.cuda.synchronize()
-            kt["score_select"].append(evs[0].elapsed_time(evs[1]))
-            kt["sparse_decode"].append(evs[1].elapsed_time(evs[2]))
-            kt["combine"].append(evs[2].elapsed_time(evs[3]))
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            ev[0].record()
+            if args.path == "fused":
+                layer_step(w, L, p, pos, path="fused")
+                ev[1].record()
+            else:
+                sba.sba_append_kv(c, li.k_new, li.v_new, pos)
+                ev[1].record()
+                if w.scorer == "gate":
+                    sba.sba_update_descriptors(c, pos, w.append_tokens, li.Wq, li.Wk)
+                else:
+                    sba.sba_update_descriptors(c, pos, w.append_tokens)
+                ev[2].record()
+                sba.sba_score_select(c, li.q, p, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, bufs.ws)
+                ev[3].record()
+                sba.sba_sparse_decode(c, li.q, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, w.scale, bufs.o_part,
+                                      bufs.lse_part)
+                ev[4].record()
+                sba.sba_combine(bufs.o_part, bufs.lse_part, bufs.out, bufs.lse)
+                ev[5].record()
+            rec.append(ev)
+        torch.cuda.synchronize()
+        for ev in rec:
+            for i, k in enumerate(names):
+                kt[k].append(ev[i].elapsed_time(ev[i + 1]))
     kmean = {k: statistics.mean(v) for k, v in kt.items()}
-    alg = {"sparse_decode": kv_bytes_layer, "score_select": desc_bytes_layer}
+    if args.path == "fused":
+        alg = {"decode_step": per_layer}
+    else:
+        alg = {"sparse_decode": kv_bytes_layer, "score_select": desc_bytes_layer}
     dom = max(alg, key=lambda k: kmean[k])
     hbm, peak_kind = peaks()
     achieved = alg[dom] / (kmean[dom] * 1e-3) / 1e9
@@ -339,7 +371,7 @@ def native(args, rank, world, local):
                 qd[i].copy_(qh[i], non_blocking=True)
                 kd[i].copy_(kh[i], non_blocking=True)
                 vd[i].copy_(vh[i], non_blocking=True)
-                layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i])
+                layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i], path=args.path)
                 oh[i].copy_(L["bufs"].out, non_blocking=True)
 
         for _ in range(2):
@@ -385,18 +417,21 @@ def native(args, rank, world, local):
             "workload": w.name, "batch": w.B, "layers": n_layers, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
             "block": w.b, "context": [min(lens), max(lens)], "blocks_selected_per_group": n_max,
             "scorer": w.scorer, "paged": w.paged, "append_tokens_per_step": w.append_tokens,
-            "num_splits": splits, "counted_bytes_per_step": step_bytes,
+            "num_splits": splits, "cluster_ctas": sba.sba_decode_step_cluster(layers[0]["c"], p),
+            "counted_bytes_per_step": step_bytes,
             "kv_bytes_per_layer": kv_bytes_layer, "desc_bytes_per_layer": desc_bytes_layer,
             "l2": (f"L2 flushed between steps (512 MB write, outside the timed events); step footprint "
                    f"{footprint / 1e6:.0f} MB" if flush else
                    f"inputs larger than L2: {footprint / 1e6:.0f} MB per step vs {l2 / 1e6:.0f} MB L2"),
             "graph": "one CUDA graph per step, programmatic dependent launch between kernels",
+            "path": ("one fused sba_decode_step launch per layer (thread-block clusters)" if args.path == "fused"
+                     else "five C-ABI calls per layer"),
             "parallelism": f"replicas x{world} (independent batches, no collective)",
         },
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": KERNELS_PER_LAYER * n_layers * args.steps,
+        "gpu_launches": KERNELS_PER_LAYER[args.path] * n_layers * args.steps,
         "clocks": clk,
     }
     del graph

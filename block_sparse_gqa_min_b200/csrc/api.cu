@@ -161,4 +161,43 @@ int sba_combine(const float* o_part, const float* lse_part, int32_t B, int32_t H
                                        static_cast<cudaStream_t>(stream)));
 }
 
+int sba_fold_gate(const sba_gate* g, float* A, void* stream) {
+    if (!g || !g->Wq || !g->Wk || !A || g->dg < 1 || g->dg > 256) return SBA_ERR_INVALID_ARG;
+    return after_launch(launch_fold_gate(g->Wq, g->Wk, g->dg, A, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t sba_decode_step_cluster(const sba_cache* c, const sba_select_params* p) {
+    if (check_cache(c) != SBA_OK || check_params(p) != SBA_OK) return 0;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return step_cluster_size(*c, *p, sms);
+}
+
+int sba_decode_step(const sba_cache* c, const void* q, const void* k_new, const void* v_new, const int32_t* pos_start,
+                    int32_t n_new, const float* gate_A, const sba_select_params* p, float softmax_scale, void* out,
+                    int32_t out_dtype, float* lse_out, int32_t* sel_idx, int32_t* sel_cnt, float* gate_bias,
+                    int32_t n_max, void* stream) {
+    int rc = check_cache(c);
+    if (rc != SBA_OK) return rc;
+    rc = check_params(p);
+    if (rc != SBA_OK) return rc;
+    if (!q || !out || !aligned16(q) || n_new < 0) return SBA_ERR_INVALID_ARG;
+    if (out_dtype != SBA_OUT_F32 && out_dtype != SBA_OUT_BF16) return SBA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return SBA_ERR_INVALID_ARG;
+    if (n_new > 0 && (!k_new || !v_new || !pos_start || !aligned16(k_new) || !aligned16(v_new)))
+        return SBA_ERR_INVALID_ARG;
+    if (p->scorer == SBA_SCORER_QUEST && !c->desc) return SBA_ERR_INVALID_ARG;
+    if (p->scorer == SBA_SCORER_GATE && (!c->kg || !gate_A)) return SBA_ERR_INVALID_ARG;
+    const int n_need = num_selected((c->max_len + c->b - 1) / c->b, *p);
+    if ((sel_idx || gate_bias) && n_max < n_need) return SBA_ERR_INVALID_ARG;
+    if (c->B > 65535 || c->H_kv > 65535) return SBA_ERR_UNSUPPORTED;
+    const int C = sba_decode_step_cluster(c, p);
+    if (C < 1) return SBA_ERR_UNSUPPORTED;
+    return after_launch(launch_decode_step(*c, q, k_new, v_new, pos_start, n_new, gate_A, *p, softmax_scale, out,
+                                           out_dtype, lse_out, sel_idx, sel_cnt,
+                                           p->scorer == SBA_SCORER_GATE ? gate_bias : nullptr, n_max, C,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -27,16 +27,15 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "decode_tile.cuh"
 #include "launch.cuh"
 
 namespace sba {
 
 namespace {
 
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = kDecodeConsumerWarps;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 struct DecodeArgs {
     const int32_t* seq_lens;
@@ -54,27 +53,15 @@ struct DecodeArgs {
     float* lse_part;
 };
 
-struct StageInfo {
-    int j;      // logical block
-    int valid;  // valid tokens in the block
-    int ok;     // 1 if the tiles were loaded
-    int pad;
-};
-
 template <int kBlk>
 struct Smem {
-    static constexpr int kHalf = kBlk * 128;    // one 64-channel half of a tile, bytes
-    static constexpr int kStage = 4 * kHalf;    // K0 K1 V0 V1
+    static constexpr int kHalf = TileGeom<kBlk>::kHalf;
+    static constexpr int kStage = TileGeom<kBlk>::kStage;
     static constexpr int kStages = kBlk == 64 ? 6 : 3;
     static constexpr int kMerge = kConsumerWarps * 16 * kHeadDim * 4 + kConsumerWarps * 16 * 2 * 4;
     static constexpr int kBars = 2 * kStages * 8 + kStages * (int)sizeof(StageInfo);
     static constexpr int kBytes = kStages * kStage + kMerge + kBars + 1024;  // + alignment slack
 };
-
-__device__ __forceinline__ uint32_t swz(uint32_t half_base, int row, int chunk) {
-    // 128-byte TMA swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
-    return half_base + row * 128 + ((chunk ^ (row & 7)) << 4);
-}
 
 template <int kBlk>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -82,8 +69,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                          DecodeArgs a) {
     using S = Smem<kBlk>;
     constexpr int kStages = S::kStages;
-    constexpr int T = kBlk / kConsumerWarps;  // tokens per consumer warp per block (16 or 32)
-    constexpr int NT = T / 8;                 // 8-token MMA n-tiles per warp
     extern __shared__ uint8_t dyn_raw[];
     uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     float* merge_o = reinterpret_cast<float*>(dyn + kStages * S::kStage);          // [4][16][128]
@@ -156,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         inf.j = j;
                         inf.valid = page >= 0 ? min(kBlk, len - j * kBlk) : 0;
                         inf.ok = page >= 0;
-                        inf.pad = 0;
+                        inf.pos = i;
                         info[st] = inf;
                         if (page >= 0) {
                             uint8_t* base = dyn + st * S::kStage;
@@ -176,180 +161,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------ consumers -----------------------------
-        const int r = lane >> 2;         // MMA row of this thread (and r + 8)
-        const int cq = (lane & 3) * 2;   // column pair inside an 8-wide tile
-        // Q as A fragments: rows = query heads of the group (zero past G)
+        const int r = lane >> 2;
         uint32_t qa[8][4];
-        {
-            const __nv_bfloat16* qb = a.q + ((int64_t)s * a.H_q + h * G) * kHeadDim;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const int c0 = ks * 16 + cq;
-                qa[ks][0] = r < G ? *reinterpret_cast<const uint32_t*>(qb + r * kHeadDim + c0) : 0u;
-                qa[ks][1] = r + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (r + 8) * kHeadDim + c0) : 0u;
-                qa[ks][2] = r < G ? *reinterpret_cast<const uint32_t*>(qb + r * kHeadDim + c0 + 8) : 0u;
-                qa[ks][3] = r + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (r + 8) * kHeadDim + c0 + 8) : 0u;
-            }
-        }
+        load_q_frags(qa, a.q + ((int64_t)s * a.H_q + h * G) * kHeadDim, G, lane);
         const float* bias_r = (a.gate_bias && r < G) ? a.gate_bias + ((int64_t)s * a.H_q + h * G + r) * a.n_max + i0 : nullptr;
         const float* bias_r8 =
             (a.gate_bias && r + 8 < G) ? a.gate_bias + ((int64_t)s * a.H_q + h * G + r + 8) * a.n_max + i0 : nullptr;
-
-        float o[16][4];
-#pragma unroll
-        for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-        float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows r, r+8
-        float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
-        const int tok0 = warp * T;
-
+        DecodeState dst;
+        decode_state_init(dst);
         for (int i = 0; i < nb; ++i) {
             const int st = i % kStages;
             if (!mbar_wait(&full[st], (i / kStages) & 1, a.status)) break;
             const StageInfo inf = info[st];
-            const uint32_t kb = smem_u32(dyn + st * S::kStage);
-            const uint32_t vb = kb + 2 * S::kHalf;
-            if (inf.ok && tok0 < inf.valid) {
-                if (inf.valid < tok0 + T) {
-                    // rows past len may hold anything: zero this warp's invalid V rows so 0*garbage cannot appear
-                    uint8_t* vrow = dyn + st * S::kStage + 2 * S::kHalf;
-                    for (int e = lane; e < (tok0 + T - inf.valid) * 16; e += 32) {
-                        const int row = inf.valid + e / 16, ch = e % 16;
-                        *reinterpret_cast<uint4*>(vrow + (ch >> 3) * S::kHalf + row * 128 + ((ch & 7) << 4)) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    __syncwarp();
-                }
-                // ---- S = Q K^T (16 x T) ----
-                float sc[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-                    const int row = tok0 + nt * 8 + (lane & 7);
-#pragma unroll
-                    for (int kp = 0; kp < 4; ++kp) {
-                        const int chunk = 4 * kp + (lane >> 3);
-                        uint32_t b0, b1, b2, b3;
-                        ldmatrix_x4(swz(kb + (chunk >> 3) * S::kHalf, row, chunk & 7), b0, b1, b2, b3);
-                        mma_bf16_16816(sc[nt], qa[2 * kp], b0, b1);
-                        mma_bf16_16816(sc[nt], qa[2 * kp + 1], b2, b3);
-                    }
-                }
-                // ---- scale, log-gate, mask, online softmax (base 2) ----
+            if (inf.ok) {
                 const float g0 = bias_r ? __ldg(bias_r + i) * kLog2e : 0.f;
                 const float g1 = bias_r8 ? __ldg(bias_r8 + i) * kLog2e : 0.f;
-                float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int t = tok0 + nt * 8 + cq;
-                    const bool v0 = t < inf.valid, v1 = t + 1 < inf.valid;
-                    sc[nt][0] = v0 ? fmaf(sc[nt][0], a.scale_log2, g0) : -INFINITY;
-                    sc[nt][1] = v1 ? fmaf(sc[nt][1], a.scale_log2, g0) : -INFINITY;
-                    sc[nt][2] = v0 ? fmaf(sc[nt][2], a.scale_log2, g1) : -INFINITY;
-                    sc[nt][3] = v1 ? fmaf(sc[nt][3], a.scale_log2, g1) : -INFINITY;
-                    mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
-                    mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
-                }
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-                const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-                const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-                const float al0 = exp2f(m0 - u0), al1 = exp2f(m1 - u1);
-                m0 = n0;
-                m1 = n1;
-                l0 *= al0;
-                l1 *= al1;
-                if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
-#pragma unroll
-                    for (int n = 0; n < 16; ++n) {
-                        o[n][0] *= al0;
-                        o[n][1] *= al0;
-                        o[n][2] *= al1;
-                        o[n][3] *= al1;
-                    }
-                }
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    sc[nt][0] = exp2f(sc[nt][0] - u0);
-                    sc[nt][1] = exp2f(sc[nt][1] - u0);
-                    sc[nt][2] = exp2f(sc[nt][2] - u1);
-                    sc[nt][3] = exp2f(sc[nt][3] - u1);
-                    l0 += sc[nt][0] + sc[nt][1];
-                    l1 += sc[nt][2] + sc[nt][3];
-                }
-                // ---- O += P V (P as bf16 hi + lo) ----
-#pragma unroll
-                for (int kt = 0; kt < NT / 2; ++kt) {
-                    uint32_t ph[4], pl[4];
-                    const float* p0 = sc[2 * kt];
-                    const float* p1 = sc[2 * kt + 1];
-                    const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 hi = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
-                        const float2 hf = __bfloat1622float2(hi);
-                        const __nv_bfloat162 lo = __floats2bfloat162_rn(pv[2 * e] - hf.x, pv[2 * e + 1] - hf.y);
-                        ph[e] = *reinterpret_cast<const uint32_t*>(&hi);
-                        pl[e] = *reinterpret_cast<const uint32_t*>(&lo);
-                    }
-                    const int row = tok0 + kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-                    for (int np = 0; np < 8; ++np) {
-                        const int chunk = 2 * np + (lane >> 4);
-                        uint32_t b0, b1, b2, b3;
-                        ldmatrix_x4_trans(swz(vb + (chunk >> 3) * S::kHalf, row, chunk & 7), b0, b1, b2, b3);
-                        mma_bf16_16816(o[2 * np], ph, b0, b1);
-                        mma_bf16_16816(o[2 * np], pl, b0, b1);
-                        mma_bf16_16816(o[2 * np + 1], ph, b2, b3);
-                        mma_bf16_16816(o[2 * np + 1], pl, b2, b3);
-                    }
-                }
+                decode_block<kBlk>(dst, qa, dyn + st * S::kStage, inf.valid, g0, g1, a.scale_log2, warp, lane);  // slot = warp
             }
             // release the stage (generic-proxy writes ordered before the next TMA write)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
-        // ---- per-warp results to shared memory ----
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-        float* mo = merge_o + warp * 16 * kHeadDim;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            *reinterpret_cast<float2*>(mo + r * kHeadDim + n * 8 + cq) = make_float2(o[n][0], o[n][1]);
-            *reinterpret_cast<float2*>(mo + (r + 8) * kHeadDim + n * 8 + cq) = make_float2(o[n][2], o[n][3]);
-        }
-        if ((lane & 3) == 0) {
-            merge_ml[(warp * 16 + r) * 2] = m0;
-            merge_ml[(warp * 16 + r) * 2 + 1] = l0;
-            merge_ml[(warp * 16 + r + 8) * 2] = m1;
-            merge_ml[(warp * 16 + r + 8) * 2 + 1] = l1;
-        }
+        decode_state_store(dst, merge_o, merge_ml, warp, lane);
     }
     __syncthreads();
     // ---- merge the four consumer warps; 128 threads = 128 channels ----
     if (tid < kHeadDim) {
         const int ch = tid;
         for (int row = 0; row < G; ++row) {
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_ml[(w * 16 + row) * 2]);
-            float osum = 0.f, lsum = 0.f;
-            if (M > -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = merge_ml[(w * 16 + row) * 2];
-                    const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                    lsum += f * merge_ml[(w * 16 + row) * 2 + 1];
-                    osum += f * merge_o[(w * 16 + row) * kHeadDim + ch];
-                }
-            }
+            float o, lse;
+            merge_warps(merge_o, merge_ml, row, ch, o, lse);
             const int64_t orow = ((int64_t)s * a.H_q + h * G + row) * a.num_splits + sp;
-            a.o_part[orow * kHeadDim + ch] = lsum > 0.f ? osum / lsum : 0.f;
-            if (ch == 0) a.lse_part[orow] = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
+            a.o_part[orow * kHeadDim + ch] = o;
+            if (ch == 0) a.lse_part[orow] = lse;
         }
     }
 }
@@ -396,8 +241,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+}  // namespace
+
 // 2-D view [rows = num_pages*H_kv*b][128] bf16 of a K or V cache; box = 64 channels x b rows.
-bool make_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk) {
+bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
@@ -409,11 +256,13 @@ bool make_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <int kBlk>
 int launch_decode_blk(const sba_cache& c, const DecodeArgs& a, cudaStream_t stream) {
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
-    if (!make_tmap(&tk, c.k, rows, kBlk) || !make_tmap(&tv, c.v, rows, kBlk)) return SBA_ERR_CUDA;
+    if (!make_kv_tmap(&tk, c.k, rows, kBlk) || !make_kv_tmap(&tv, c.v, rows, kBlk)) return SBA_ERR_CUDA;
     const int smem = Smem<kBlk>::kBytes;
     if (allow_smem<sparse_decode_kernel<kBlk>>(smem) != SBA_OK) return SBA_ERR_CUDA;
     dim3 grid(a.num_splits, c.H_kv, c.B);

@@ -1,0 +1,217 @@
+// Per-block attention math of the sparse decode, shared by the split-KV
+// decode kernel and the fused decode-step kernel.
+//
+// A consumer warp owns T = b/4 tokens of every K/V block staged in shared
+// memory (128-byte TMA swizzle, two 64-channel halves per tensor).  The G query
+// heads of the group are the 16 rows of bf16 tensor-core tiles (m16n8k16,
+// fp32 accumulate, rows past G are zero): S = Q K^T, online base-2 softmax with
+// the optional log-gate ("SAS ...", Method: softmax(q K^T + log g) V), then
+// O += P V with P split into bf16 hi + lo parts (about 16 mantissa bits).
+#pragma once
+
+#include "common.cuh"
+
+namespace sba {
+
+constexpr int kDecodeConsumerWarps = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int kBlk>
+struct TileGeom {
+    static constexpr int kHalf = kBlk * 128;   // one 64-channel half of a tile, bytes
+    static constexpr int kStage = 4 * kHalf;   // K0 K1 V0 V1
+    static constexpr int T = kBlk / kDecodeConsumerWarps;  // tokens per consumer warp
+    static constexpr int NT = T / 8;                        // 8-token MMA n-tiles per warp
+};
+
+struct StageInfo {
+    int j;      // logical block
+    int valid;  // valid tokens in the block
+    int ok;     // 1 if the tiles were loaded
+    int pos;    // position of the block in the selection
+};
+
+__device__ __forceinline__ uint32_t swz(uint32_t half_base, int row, int chunk) {
+    // 128-byte TMA swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
+    return half_base + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+struct DecodeState {
+    float o[16][4];
+    float m0, m1;  // running max (log2 units) of rows r, r+8
+    float l0, l1;  // this thread's partial sums of rows r, r+8
+};
+
+__device__ __forceinline__ void decode_state_init(DecodeState& st) {
+#pragma unroll
+    for (int n = 0; n < 16; ++n) st.o[n][0] = st.o[n][1] = st.o[n][2] = st.o[n][3] = 0.f;
+    st.m0 = st.m1 = -INFINITY;
+    st.l0 = st.l1 = 0.f;
+}
+
+// Q of the group (rows = query heads, zero past G) as m16n8k16 A fragments.
+__device__ __forceinline__ void load_q_frags(uint32_t (&qa)[8][4], const __nv_bfloat16* qb, int G, int lane) {
+    const int r = lane >> 2, cq = (lane & 3) * 2;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        const int c0 = ks * 16 + cq;
+        qa[ks][0] = r < G ? *reinterpret_cast<const uint32_t*>(qb + r * kHeadDim + c0) : 0u;
+        qa[ks][1] = r + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (r + 8) * kHeadDim + c0) : 0u;
+        qa[ks][2] = r < G ? *reinterpret_cast<const uint32_t*>(qb + r * kHeadDim + c0 + 8) : 0u;
+        qa[ks][3] = r + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (r + 8) * kHeadDim + c0 + 8) : 0u;
+    }
+}
+
+// One staged block: the T tokens of token slot `slot` (0..3).  `stage` is the generic pointer of
+// the stage, `valid` the block's valid token count, g0/g1 the log-gates of
+// rows r and r+8 (already in log2 units).
+template <int kBlk>
+__device__ __forceinline__ void decode_block(DecodeState& st, const uint32_t (&qa)[8][4], uint8_t* stage, int valid,
+                                             float g0, float g1, float scale_log2, int slot, int lane) {
+    using TG = TileGeom<kBlk>;
+    constexpr int T = TG::T, NT = TG::NT;
+    const int tok0 = slot * T;  // this warp's tokens: slot 0..3 of the block
+    if (tok0 >= valid) return;
+    const int cq = (lane & 3) * 2;
+    const uint32_t kb = smem_u32(stage);
+    const uint32_t vb = kb + 2 * TG::kHalf;
+    if (valid < tok0 + T) {
+        // rows past len may hold anything: zero this warp's invalid V rows so 0*garbage cannot appear
+        uint8_t* vrow = stage + 2 * TG::kHalf;
+        for (int e = lane; e < (tok0 + T - valid) * 16; e += 32) {
+            const int row = valid + e / 16, ch = e % 16;
+            *reinterpret_cast<uint4*>(vrow + (ch >> 3) * TG::kHalf + row * 128 + ((ch & 7) << 4)) =
+                make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+    }
+    // ---- S = Q K^T (16 x T) ----
+    float sc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        const int row = tok0 + nt * 8 + (lane & 7);
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {
+            const int chunk = 4 * kp + (lane >> 3);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(swz(kb + (chunk >> 3) * TG::kHalf, row, chunk & 7), b0, b1, b2, b3);
+            mma_bf16_16816(sc[nt], qa[2 * kp], b0, b1);
+            mma_bf16_16816(sc[nt], qa[2 * kp + 1], b2, b3);
+        }
+    }
+    // ---- scale, log-gate, mask, online softmax (base 2) ----
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int t = tok0 + nt * 8 + cq;
+        const bool v0 = t < valid, v1 = t + 1 < valid;
+        sc[nt][0] = v0 ? fmaf(sc[nt][0], scale_log2, g0) : -INFINITY;
+        sc[nt][1] = v1 ? fmaf(sc[nt][1], scale_log2, g0) : -INFINITY;
+        sc[nt][2] = v0 ? fmaf(sc[nt][2], scale_log2, g1) : -INFINITY;
+        sc[nt][3] = v1 ? fmaf(sc[nt][3], scale_log2, g1) : -INFINITY;
+        mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+        mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
+    const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
+    const float al0 = exp2f(st.m0 - u0), al1 = exp2f(st.m1 - u1);
+    st.m0 = n0;
+    st.m1 = n1;
+    st.l0 *= al0;
+    st.l1 *= al1;
+    if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            st.o[n][0] *= al0;
+            st.o[n][1] *= al0;
+            st.o[n][2] *= al1;
+            st.o[n][3] *= al1;
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        sc[nt][0] = exp2f(sc[nt][0] - u0);
+        sc[nt][1] = exp2f(sc[nt][1] - u0);
+        sc[nt][2] = exp2f(sc[nt][2] - u1);
+        sc[nt][3] = exp2f(sc[nt][3] - u1);
+        st.l0 += sc[nt][0] + sc[nt][1];
+        st.l1 += sc[nt][2] + sc[nt][3];
+    }
+    // ---- O += P V (P as bf16 hi + lo) ----
+#pragma unroll
+    for (int kt = 0; kt < NT / 2; ++kt) {
+        uint32_t ph[4], pl[4];
+        const float* p0 = sc[2 * kt];
+        const float* p1 = sc[2 * kt + 1];
+        const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
+            const float2 hf = __bfloat1622float2(hi);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(pv[2 * e] - hf.x, pv[2 * e + 1] - hf.y);
+            ph[e] = *reinterpret_cast<const uint32_t*>(&hi);
+            pl[e] = *reinterpret_cast<const uint32_t*>(&lo);
+        }
+        const int row = tok0 + kt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int np = 0; np < 8; ++np) {
+            const int chunk = 2 * np + (lane >> 4);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4_trans(swz(vb + (chunk >> 3) * TG::kHalf, row, chunk & 7), b0, b1, b2, b3);
+            mma_bf16_16816(st.o[2 * np], ph, b0, b1);
+            mma_bf16_16816(st.o[2 * np], pl, b0, b1);
+            mma_bf16_16816(st.o[2 * np + 1], ph, b2, b3);
+            mma_bf16_16816(st.o[2 * np + 1], pl, b2, b3);
+        }
+    }
+}
+
+// This warp's (max, sum, O) rows to shared memory: merge_o [warps][16][128],
+// merge_ml [warps][16][2].
+__device__ __forceinline__ void decode_state_store(DecodeState& st, float* merge_o, float* merge_ml, int warp,
+                                                   int lane) {
+    const int r = lane >> 2, cq = (lane & 3) * 2;
+    st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, 1);
+    st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, 2);
+    st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, 1);
+    st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, 2);
+    float* mo = merge_o + warp * 16 * kHeadDim;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        *reinterpret_cast<float2*>(mo + r * kHeadDim + n * 8 + cq) = make_float2(st.o[n][0], st.o[n][1]);
+        *reinterpret_cast<float2*>(mo + (r + 8) * kHeadDim + n * 8 + cq) = make_float2(st.o[n][2], st.o[n][3]);
+    }
+    if ((lane & 3) == 0) {
+        merge_ml[(warp * 16 + r) * 2] = st.m0;
+        merge_ml[(warp * 16 + r) * 2 + 1] = st.l0;
+        merge_ml[(warp * 16 + r + 8) * 2] = st.m1;
+        merge_ml[(warp * 16 + r + 8) * 2 + 1] = st.l1;
+    }
+}
+
+// Merge `nwarps` consumer warps' states for (row, channel): normalised O and the
+// natural-log LSE of the row (-inf and O = 0 when the row saw no token).
+__device__ __forceinline__ void merge_warps(const float* merge_o, const float* merge_ml, int row, int ch, float& o,
+                                            float& lse, int nwarps = kDecodeConsumerWarps) {
+    float M = -INFINITY;
+    for (int w = 0; w < nwarps; ++w) M = fmaxf(M, merge_ml[(w * 16 + row) * 2]);
+    float osum = 0.f, lsum = 0.f;
+    if (M > -INFINITY) {
+        for (int w = 0; w < nwarps; ++w) {
+            const float mw = merge_ml[(w * 16 + row) * 2];
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            lsum += f * merge_ml[(w * 16 + row) * 2 + 1];
+            osum += f * merge_o[(w * 16 + row) * kHeadDim + ch];
+        }
+    }
+    o = lsum > 0.f ? osum / lsum : 0.f;
+    lse = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
+}
+
+}  // namespace sba

@@ -1,0 +1,1070 @@
+// Fused decode step: append -> descriptor refresh -> block scoring -> shared
+// top-n selection -> sparse attention -> merge, in ONE launch per layer.
+//
+// Same method as the separate calls ("Rectified Sparse Attention for
+// Efficient Long-Sequence Generation", Summary and Key points; "SAS: Simple
+// Attention Sparsification ...", Method), organised for B200:
+//  - one thread-block CLUSTER of C CTAs (one CTA per SM) per (sequence, KV
+//    group); CTA r owns slice r of the blocks [0, max_blocks) for scoring and
+//    share r of the selected blocks for attention;
+//  - descriptors stream into a shared-memory ring with 1-D bulk copies (TMA
+//    engine, mbarrier completion); K/V tiles with 2-D TMA loads (128-B swizzle);
+//  - the selection is distributed: each CTA pushes the maxima of groups of its
+//    scores to its peers (distributed shared memory); every CTA derives the same
+//    lower bound T0 of the n-th score from them (k group maxima are k distinct
+//    candidates), pushes its candidates >= T0 (score, index, page) into a
+//    cluster-wide list, and ranks that short list exactly.  Scores never reach
+//    global memory;
+//  - partial (O, LSE) of the CTAs are pushed to the merging CTA of each output
+//    element; all pushes precede a cluster barrier, after which every CTA reads
+//    only its own shared memory;
+//  - the appended tokens are written by CTA 0 before the first cluster barrier,
+//    and the descriptors of the touched blocks are recomputed from the K tiles
+//    the decode stages anyway (the touched blocks are local, hence selected).
+//    When a touched block is one the step itself scores (e.g. no local
+//    blocks), CTA 0 refreshes it from global memory first and a cluster barrier
+//    orders that before the scoring.
+// No workspace: every intermediate lives in shared memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "decode_tile.cuh"
+#include "launch.cuh"
+#include "select.cuh"
+
+namespace sba {
+
+bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);  // decode.cu
+
+namespace {
+
+constexpr int kGW = kDecodeConsumerWarps;  // warps of one consumer group (4 token slots)
+constexpr int kGroups = 2;                  // consumer groups: alternate ring stages
+constexpr int kCW = kGW * kGroups;          // consumer warps
+constexpr int kThreads = (kCW + 1) * 32;
+constexpr int kProducer = kCW;
+constexpr int kMaxCluster = 16;
+constexpr int kDescBytes = 512;
+
+struct StepArgs {
+    sba_cache c;
+    const __nv_bfloat16* q;
+    const uint4* k_new;
+    const uint4* v_new;
+    const int32_t* pos_start;
+    int n_new;
+    const float* gate_A;  // [128][384]: folded gate projection
+    sba_select_params p;
+    float scale_log2;
+    void* out;
+    int out_dtype;
+    float* lse_out;
+    int32_t* sel_idx;
+    int32_t* sel_cnt;
+    float* gate_bias;
+    int n_max;
+    // shared-memory layout (bytes from the 1024-aligned base) and capacities
+    int n_stages;
+    int slice;      // blocks of [0, max_blocks) per CTA (multiple of 4)
+    int off_keys, off_pages, off_u, off_gmax, off_ckey, off_cidx, off_cpage, off_crank, off_sel, off_selp,
+        off_recv, off_bars;
+    int gcap;       // group maxima per CTA slot
+    int ccap;       // candidate slots (cluster total)
+    int sel_cap;    // words in sel / sel_page
+};
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n)); }
+
+// Reduce-scatter of NB per-block partial sums (V values each) over the 32
+// lanes: on return out[] holds, in every lane, the full sums of block
+// rs_block<NB>(lane).
+template <int NB, int V>
+__device__ __forceinline__ void reduce_scatter(float (&v)[NB][V], float (&out)[V], int lane) {
+    int n = NB;
+#pragma unroll
+    for (int m = 16; m >= (NB == 8 ? 4 : 8); m >>= 1) {
+        const bool up = (lane & m) != 0;
+        const int half = n >> 1;
+#pragma unroll
+        for (int k = 0; k < NB / 2; ++k) {
+            if (k < half) {
+#pragma unroll
+                for (int x = 0; x < V; ++x) {
+                    const float send = up ? v[k][x] : v[k + half][x];
+                    const float keep = up ? v[k + half][x] : v[k][x];
+                    v[k][x] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+        }
+        n = half;
+    }
+#pragma unroll
+    for (int x = 0; x < V; ++x) {
+        float t = v[0][x];
+        if (NB == 4) t += __shfl_xor_sync(0xffffffffu, t, 4);
+        t += __shfl_xor_sync(0xffffffffu, t, 2);
+        t += __shfl_xor_sync(0xffffffffu, t, 1);
+        out[x] = t;
+    }
+}
+
+template <int NB>
+__device__ __forceinline__ int rs_block(int lane) {
+    return NB == 8 ? (((lane >> 4) & 1) << 2) | (((lane >> 3) & 1) << 1) | ((lane >> 2) & 1)
+                   : (((lane >> 4) & 1) << 1) | ((lane >> 3) & 1);
+}
+
+// CTA 0: write the step's new tokens of (s, h) into the cache.
+__device__ void append_rows(const StepArgs& a, int s, int h, int p0, int tid) {
+    const sba_cache& c = a.c;
+    const int total = a.n_new * 32;  // per token: 16 x 16 B of K, 16 x 16 B of V
+    for (int e = tid; e < total; e += kThreads) {
+        const int tok = e >> 5, half = (e >> 4) & 1, l = e & 15;
+        const int pos = p0 + tok;
+        const int64_t page = page_of(c, s, pos / c.b, c.status);
+        if (page < 0) continue;
+        const uint4* src = (half ? a.v_new : a.k_new) + (((int64_t)s * a.n_new + tok) * c.H_kv + h) * 16 + l;
+        uint4* dst = reinterpret_cast<uint4*>(half ? c.v : c.k) + ((page * c.H_kv + h) * c.b + pos % c.b) * 16 + l;
+        *dst = __ldg(src);
+    }
+    fence_proxy_async_global();
+}
+
+// Descriptor of block j of (s, h) from global memory (threads 0..127, one
+// channel each).  Quest: min/max rows; gate: pooled -> kg = A pooled.
+template <int kScorer>
+__device__ void refresh_from_global(const StepArgs& a, int s, int h, int j, int len, float* pooled, int tid) {
+    const sba_cache& c = a.c;
+    const int64_t page = page_of(c, s, j, tid == 0 ? c.status : nullptr);
+    const int cnt = min(c.b, len - j * c.b);
+    if (page >= 0 && cnt > 0 && tid < kHeadDim) {
+        const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(c.k) + (page * c.H_kv + h) * c.b * kHeadDim;
+        float lo = INFINITY, hi = -INFINITY, sum = 0.f;
+        for (int t = 0; t < cnt; ++t) {
+            const float x = __bfloat162float(kt[t * kHeadDim + tid]);
+            lo = fminf(lo, x);
+            hi = fmaxf(hi, x);
+            sum += x;
+        }
+        if (kScorer == SBA_SCORER_QUEST) {
+            __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(c.desc) + (page * c.H_kv + h) * 2 * kHeadDim;
+            d[tid] = __float2bfloat16_rn(lo);
+            d[kHeadDim + tid] = __float2bfloat16_rn(hi);
+        } else {
+            pooled[tid] = hi;
+            pooled[kHeadDim + tid] = lo;
+            pooled[2 * kHeadDim + tid] = sum / (float)cnt;
+        }
+    }
+    if (kScorer == SBA_SCORER_GATE) {
+        __syncthreads();
+        if (page >= 0 && cnt > 0 && tid < kHeadDim) {
+            const float* Ar = a.gate_A + (int64_t)tid * 3 * kHeadDim;
+            float acc = 0.f;
+            for (int i = 0; i < 3 * kHeadDim; ++i) acc = fmaf(__ldg(Ar + i), pooled[i], acc);
+            c.kg[(page * c.H_kv + h) * kHeadDim + tid] = acc;
+        }
+        __syncthreads();
+    }
+}
+
+// Physical page of block j without reporting (speculative lookups).
+__device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
+    const int64_t p = c.block_table ? (int64_t)__ldg(c.block_table + (int64_t)s * c.max_blocks + j)
+                                    : (int64_t)s * c.max_blocks + j;
+    return (p < 0 || p >= c.num_pages) ? -1 : (int)p;
+}
+
+template <int kBlk, int kScorer, int kGM>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, StepArgs a) {
+    using TG = TileGeom<kBlk>;
+    constexpr int kChunk = 64;  // descriptors per ring fill; consecutive fills alternate consumer groups
+    constexpr int kMaxLocal = 64;
+    __shared__ uint32_t hist[256];
+    __shared__ int warp_tot[kThreads / 32];
+    __shared__ uint32_t sh[2];
+    __shared__ int misc[4];
+    __shared__ float lse_s[kMaxGroup];
+    __shared__ float lse_all[kMaxCluster * kMaxGroup];
+    __shared__ float mz_all[kMaxCluster * kMaxGroup][2];
+    __shared__ int cnt_g[kMaxCluster];    // group maxima pushed by each CTA
+    __shared__ int end_all[kMaxCluster];  // candidates each CTA pushed
+    __shared__ int local_page[kMaxLocal];
+    __shared__ __align__(16) float pooled[3 * kHeadDim];     // refresh-before-score scratch
+    __shared__ __align__(16) float pooled_b0[3 * kHeadDim];  // pushed pooled summary of B0
+
+    extern __shared__ uint8_t dyn_raw[];
+    uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
+    const int NSt = a.n_stages;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(dyn + a.off_keys);  // own slice
+    int* pages = reinterpret_cast<int*>(dyn + a.off_pages);          // own slice
+    float* u_s = reinterpret_cast<float*>(dyn + a.off_u);            // gate: [G][slice]
+    uint32_t* gmax_all = reinterpret_cast<uint32_t*>(dyn + a.off_gmax);  // [C][gcap]
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + a.off_ckey);      // [ccap]
+    int* cidx = reinterpret_cast<int*>(dyn + a.off_cidx);
+    int* cpage = reinterpret_cast<int*>(dyn + a.off_cpage);
+    int* crank = reinterpret_cast<int*>(dyn + a.off_crank);
+    int* sel = reinterpret_cast<int*>(dyn + a.off_sel);
+    int* sel_page = reinterpret_cast<int*>(dyn + a.off_selp);
+    float* recv_o = reinterpret_cast<float*>(dyn + a.off_recv);
+    uint64_t* full = reinterpret_cast<uint64_t*>(dyn + a.off_bars);
+    uint64_t* empty = full + NSt;
+    StageInfo* info = reinterpret_cast<StageInfo*>(empty + NSt);
+    // after the decode: per-warp merge area (aliases the ring)
+    float* merge_o = reinterpret_cast<float*>(dyn);
+    float* merge_ml = merge_o + kCW * 16 * kHeadDim;
+
+    const sba_cache& c = a.c;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = (int)cluster_rank(), C = (int)cluster_size();
+    const int h = blockIdx.y, s = blockIdx.z;
+    const int G = c.H_q / c.H_kv;
+    const int mb = c.max_blocks;
+    const int slice = a.slice;
+    const int j0 = min(r * slice, mb), j1 = min(j0 + slice, mb);
+
+    if (tid == 0) {
+        for (int i = 0; i < NSt; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kGW);  // one consumer group releases a stage
+        }
+        fence_mbar_init();
+    }
+    if (warp == kProducer && lane == 0) {
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_trigger();
+
+    // ---------------- shapes of this (sequence, group) ----------------
+    const int len = __ldg(c.seq_lens + s);
+    const int p0raw = a.n_new > 0 ? __ldg(a.pos_start + s) : 0;
+    if (warp == kProducer)  // speculative page ids of the slice while the lengths arrive
+        for (int j = j0 + lane; j < j1; j += 32) pages[j - j0] = page_quiet(c, s, j);
+    int N = blocks_of(len, kBlk);
+    if (N > mb) {
+        if (tid == 0 && r == 0) report(c.status, SBA_DEV_BAD_POSITION);
+        N = mb;
+    }
+    const int L = num_local(N, a.p);
+    const int n_sel = min(num_selected(N, a.p), a.sel_cap);
+    const int NC = N - L;                                               // ranked candidates [0, NC)
+    const int NSc = kScorer == SBA_SCORER_GATE ? max(N - 1, 0) : NC;   // blocks this step scores
+    const int js1 = max(j0, min(j1, NSc));                              // my scored blocks [j0, js1)
+    const int jc1 = max(j0, min(j1, NC));                               // my ranked candidates [j0, jc1)
+    const int k = n_sel - L;
+    const bool trivial = k <= 0 || k >= NC;  // take none / all of the candidates
+    for (int i = tid; i < L && i < kMaxLocal; i += kThreads) local_page[i] = page_quiet(c, s, NC + i);
+
+    int n_new = a.n_new, p0 = 0, tb0 = 1, tb1 = 0;
+    if (n_new > 0) {
+        p0 = p0raw;
+        if (p0 < 0 || (int64_t)p0 + n_new > (int64_t)mb * kBlk) {
+            if (tid == 0 && r == 0) report(c.status, SBA_DEV_BAD_POSITION);
+            n_new = 0;
+        } else {
+            tb0 = p0 / kBlk;
+            tb1 = min((p0 + n_new - 1) / kBlk, N - 1);
+        }
+    }
+    const bool touched_scored = n_new > 0 && tb0 <= tb1 && tb0 < NSc;
+
+    // ---------------- append (and, if needed, refresh before scoring) ----------------
+    if (r == 0 && n_new > 0) {
+        append_rows(a, s, h, p0, tid);
+        if (touched_scored) {
+            __syncthreads();
+            for (int j = tb0; j <= tb1; ++j) refresh_from_global<kScorer>(a, s, h, j, len, pooled, tid);
+            fence_proxy_async_global();
+        }
+    }
+    if (touched_scored) cluster_sync();
+
+    // ---------------- phase 1: score this CTA's slice ----------------
+    uint32_t fill = 0;
+    if (warp == kProducer) {
+        for (int j = j0 + lane; j < min(j1, N); j += 32)
+            if (pages[j - j0] < 0) report(c.status, SBA_DEV_BAD_PAGE);
+        const uint8_t* dbase = kScorer == SBA_SCORER_QUEST ? reinterpret_cast<const uint8_t*>(c.desc)
+                                                            : reinterpret_cast<const uint8_t*>(c.kg);
+        bool alive = true;
+        for (int cb = j0; cb < js1; cb += kChunk, ++fill) {
+            const int st = fill % NSt;
+            const int nblk = min(kChunk, js1 - cb);
+            if (lane == 0 && fill >= (uint32_t)NSt && alive)
+                alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
+            alive = __shfl_sync(0xffffffffu, alive, 0);
+            int nv = 0;
+            for (int i = lane; i < nblk; i += 32) nv += pages[cb + i - j0] >= 0;
+            nv = __reduce_add_sync(0xffffffffu, nv);
+            if (lane == 0 && alive) {
+                if (nv > 0)
+                    mbar_arrive_expect_tx(&full[st], nv * kDescBytes);
+                else
+                    mbar_arrive(&full[st]);
+            }
+            __syncwarp();
+            if (alive && nv > 0) {
+                uint8_t* stage = dyn + (size_t)st * TG::kStage;
+                for (int i = lane; i < nblk; i += 32) {
+                    const int pg = pages[cb + i - j0];
+                    if (pg >= 0)
+                        bulk_load(stage + i * kDescBytes, dbase + ((int64_t)pg * c.H_kv + h) * kDescBytes, kDescBytes,
+                                  &full[st]);
+                }
+            }
+        }
+    } else {
+        // consumers: coefficients of this lane's 16-byte chunk of a 512-byte descriptor
+        float coef[8];
+        float qg[kGM][4];  // gate: kGM = G rounded up to a power of two
+        if (kScorer == SBA_SCORER_QUEST) {
+            // chunk lane < 16: MIN row channels 8*lane..+7 (weights M = sum_qh min(q,0));
+            // lane >= 16: MAX row channels 8*(lane-16)..+7 (weights P = sum_qh max(q,0))
+            const int ch0 = (lane & 15) * 8;
+            const bool use_max = lane >= 16;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) coef[e] = 0.f;
+            for (int g = 0; g < G; ++g) {
+                const uint4 w =
+                    __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim + ch0));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = bf16_lo(ws[e]), x1 = bf16_hi(ws[e]);
+                    coef[2 * e] += use_max ? fmaxf(x0, 0.f) : fminf(x0, 0.f);
+                    coef[2 * e + 1] += use_max ? fmaxf(x1, 0.f) : fminf(x1, 0.f);
+                }
+            }
+        } else {
+            // gate: lane owns channels 4*lane..4*lane+3 of the fp32 gate key
+#pragma unroll
+            for (int g = 0; g < kGM; ++g) {
+                if (g < G) {
+                    const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim +
+                                                                        4 * lane));
+                    qg[g][0] = bf16_lo(w.x);
+                    qg[g][1] = bf16_hi(w.x);
+                    qg[g][2] = bf16_lo(w.y);
+                    qg[g][3] = bf16_hi(w.y);
+                } else {
+                    qg[g][0] = qg[g][1] = qg[g][2] = qg[g][3] = 0.f;
+                }
+            }
+        }
+        bool alive = true;
+        const int grp = warp / kGW, gw = warp % kGW;  // consumer group, warp within the group
+        for (int cb = j0; cb < js1; cb += kChunk, ++fill) {
+            if ((int)(fill & 1) != grp) continue;  // the other group's stage
+            const int st = fill % NSt;
+            if (alive) alive = mbar_wait(&full[st], (fill / NSt) & 1, c.status);
+            const int nblk = min(kChunk, js1 - cb);
+            const uint8_t* stage = dyn + (size_t)st * TG::kStage;
+            if (kScorer == SBA_SCORER_QUEST) {
+                for (int g8 = gw * 8; g8 < nblk; g8 += kGW * 8) {
+                    float part[8][1];
+#pragma unroll
+                    for (int b8 = 0; b8 < 8; ++b8) {
+                        part[b8][0] = 0.f;
+                        if (g8 + b8 < nblk && alive) {
+                            const uint4 w = *reinterpret_cast<const uint4*>(stage + (g8 + b8) * kDescBytes + lane * 16);
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                            float acc = 0.f;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                acc = fmaf(coef[2 * e], bf16_lo(ws[e]), acc);
+                                acc = fmaf(coef[2 * e + 1], bf16_hi(ws[e]), acc);
+                            }
+                            part[b8][0] = acc;
+                        }
+                    }
+                    float tot[1];
+                    reduce_scatter<8, 1>(part, tot, lane);
+                    const int i = g8 + rs_block<8>(lane);
+                    if ((lane & 3) == 0 && i < nblk) {
+                        const int jl = cb + i - j0;
+                        keys[jl] = pages[jl] >= 0 ? orderable_key(tot[0]) : 0u;
+                    }
+                }
+            } else {
+                for (int g4 = gw * 4; g4 < nblk; g4 += kGW * 4) {
+                    float part[4][kGM];
+#pragma unroll
+                    for (int b4 = 0; b4 < 4; ++b4) {
+                        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (g4 + b4 < nblk && alive)
+                            w = *reinterpret_cast<const float4*>(stage + (g4 + b4) * kDescBytes + lane * 16);
+#pragma unroll
+                        for (int g = 0; g < kGM; ++g) {
+                            float acc = qg[g][0] * w.x;
+                            acc = fmaf(qg[g][1], w.y, acc);
+                            acc = fmaf(qg[g][2], w.z, acc);
+                            acc = fmaf(qg[g][3], w.w, acc);
+                            part[b4][g] = acc;
+                        }
+                    }
+                    float tot[kGM];
+                    reduce_scatter<4, kGM>(part, tot, lane);
+                    const int i = g4 + rs_block<4>(lane);
+                    if ((lane & 7) == 0 && i < nblk) {
+                        const int jl = cb + i - j0;
+                        const bool ok = pages[jl] >= 0;
+#pragma unroll
+                        for (int g = 0; g < kGM; ++g)
+                            if (g < G) u_s[g * slice + jl] = ok ? tot[g] : -INFINITY;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+    }
+    __syncthreads();
+
+    // ---------------- phase 2: distributed selection ----------------
+    if (kScorer == SBA_SCORER_GATE) {
+        // per-head (max, sum exp(u - max)) over this CTA's scored blocks, pushed to every CTA
+        for (int g = warp; g < G; g += kThreads / 32) {
+            float m = -INFINITY;
+            for (int i = lane; i < js1 - j0; i += 32) m = fmaxf(m, u_s[g * slice + i]);
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            float z = 0.f;
+            if (m > -INFINITY)
+                for (int i = lane; i < js1 - j0; i += 32) z += expf(u_s[g * slice + i] - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            for (int p = lane; p < C; p += 32) {
+                st_peer_f32(peer_addr(&mz_all[r * G + g][0], p), m);
+                st_peer_f32(peer_addr(&mz_all[r * G + g][1], p), z);
+            }
+        }
+        cluster_sync();  // gate round: every CTA's softmax partials pushed
+        if (tid < G) {
+            float M = -INFINITY;
+            for (int p = 0; p < C; ++p) M = fmaxf(M, mz_all[p * G + tid][0]);
+            float Z = 0.f;
+            if (M > -INFINITY)
+                for (int p = 0; p < C; ++p) {
+                    const float m = mz_all[p * G + tid][0];
+                    if (m > -INFINITY) Z += mz_all[p * G + tid][1] * expf(m - M);
+                }
+            lse_s[tid] = M > -INFINITY ? M + logf(Z) : -INFINITY;
+        }
+        __syncthreads();
+        // group score of my ranked blocks: sum over the group of g = exp(u - LSE)
+        for (int j = j0 + tid; j < jc1; j += kThreads) {
+            float sc = 0.f;
+            for (int g = 0; g < G; ++g) sc += expf(u_s[g * slice + (j - j0)] - lse_s[g]);
+            keys[j - j0] = pages[j - j0] >= 0 ? orderable_key(sc) : 0u;
+        }
+        __syncthreads();
+    }
+    // group size: the largest power of two in [4, 128] leaving >= 2k groups
+    int gs = 128;
+    if (!trivial)
+        while (gs > 4 && (NC + gs - 1) / gs < 2 * k) gs >>= 1;
+    const int lpg = gs / 4;
+    const int nown = jc1 - j0;                 // my ranked candidates
+    const int ngr = (nown + gs - 1) / gs;      // my groups
+    if (!trivial) {
+        // maxima of my groups (four keys per thread, groups of lpg lanes), pushed to every CTA
+        const uint4* kv = reinterpret_cast<const uint4*>(keys);
+        const int nv = (nown + 3) / 4;
+        for (int v0 = warp * 32; v0 < nv; v0 += kThreads) {
+            const int v = v0 + lane;
+            uint32_t m = 0;
+            if (v < nv) {
+                const uint4 q = kv[v];
+                const int j = 4 * v;
+                m = max(max(j < nown ? q.x : 0u, j + 1 < nown ? q.y : 0u),
+                        max(j + 2 < nown ? q.z : 0u, j + 3 < nown ? q.w : 0u));
+            }
+            for (int o = 1; o < lpg; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((lane & (lpg - 1)) == 0 && v < nv) {
+                const int g = v / lpg;
+                for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(gmax_all + r * a.gcap + g, p), m);
+            }
+        }
+        for (int p = tid; p < C; p += kThreads) st_peer_u32(peer_addr(&cnt_g[r], p), (uint32_t)ngr);
+    }
+    cluster_sync();  // every CTA's group maxima pushed
+    if (!trivial) {
+        // T0 = smallest group maximum with fewer than k group maxima above it (a valid lower
+        // bound of the n-th score only when there are >= k groups; otherwise take T0 = 0).
+        // The maxima are first packed contiguously (into the crank scratch), then every
+        // thread ranks its maxima against all of them with independent partial counts.
+        uint32_t* gm = reinterpret_cast<uint32_t*>(crank);
+        int ng_total = 0;
+        for (int p = 0; p < C; ++p) ng_total += cnt_g[p];
+        const bool bound = ng_total >= k && ng_total <= a.ccap;
+        if (bound)
+            for (int p = 0, off = 0; p < C; off += cnt_g[p], ++p)
+                for (int g = tid; g < cnt_g[p]; g += kThreads) gm[off + g] = gmax_all[p * a.gcap + g];
+        if (tid == 0) misc[0] = bound ? -1 : 0;
+        __syncthreads();
+        if (bound)
+            for (int g0 = warp * 32; g0 < ng_total; g0 += kThreads) {
+                const int g = g0 + lane;
+                uint32_t cand = 0xffffffffu;
+                if (g < ng_total) {
+                    const uint32_t x = gm[g];
+                    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+                    int t = 0;
+                    for (; t + 4 <= ng_total; t += 4) {
+                        a0 += gm[t] > x;
+                        a1 += gm[t + 1] > x;
+                        a2 += gm[t + 2] > x;
+                        a3 += gm[t + 3] > x;
+                    }
+                    for (; t < ng_total; ++t) a0 += gm[t] > x;
+                    if (a0 + a1 + a2 + a3 < k) cand = x;
+                }
+                cand = __reduce_min_sync(0xffffffffu, cand);
+                if (lane == 0 && cand != 0xffffffffu) atomicMin(reinterpret_cast<unsigned*>(&misc[0]), cand);
+            }
+        __syncthreads();
+        const uint32_t T0 = (uint32_t)misc[0];
+        // my candidates >= T0 go to my slots [r*cs, r*cs + cs) of every CTA's list,
+        // with their count; a count above cs marks an overflow
+        const int cs = a.ccap / C;
+        if (tid == 0) misc[2] = 0;
+        __syncthreads();
+        for (int i0 = warp * 32; i0 < nown; i0 += kThreads) {
+            const int i = i0 + lane;
+            const bool pass = i < nown && keys[i] >= T0;
+            const unsigned bal = __ballot_sync(0xffffffffu, pass);
+            int off = 0;
+            if (lane == 0 && bal) off = atomicAdd(&misc[2], __popc(bal));
+            off = __shfl_sync(0xffffffffu, off, 0);
+            if (pass) {
+                const int pos = off + __popc(bal & ((1u << lane) - 1u));
+                if (pos < cs) {
+                    const int slot = r * cs + pos;
+                    const uint32_t kk = keys[i];
+                    const int pg = pages[i];
+                    for (int p = 0; p < C; ++p) {
+                        st_peer_u32(peer_addr(ckey + slot, p), kk);
+                        st_peer_u32(peer_addr(cidx + slot, p), (uint32_t)(j0 + i));
+                        st_peer_u32(peer_addr(cpage + slot, p), (uint32_t)pg);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        for (int p = tid; p < C; p += kThreads) st_peer_u32(peer_addr(&end_all[r], p), (uint32_t)misc[2]);
+    }
+    cluster_sync();  // every candidate pushed
+    if (trivial) {
+        const int first = k <= 0 ? NC : 0;
+        for (int i = tid; i < N - first; i += kThreads) {
+            sel[i] = first + i;
+            sel_page[i] = first + i >= NC ? local_page[first + i - NC] : -1;
+        }
+    } else {
+        // the per-source slots, compacted into [0, m) of the idle ring, unless a source overflowed
+        const int cs = a.ccap / C;
+        bool overflow = false;
+        int m = 0;
+        for (int p = 0; p < C; ++p) {
+            overflow |= end_all[p] > cs;
+            m += min(end_all[p], cs);
+        }
+        uint32_t* ck = reinterpret_cast<uint32_t*>(dyn);
+        int* ci = reinterpret_cast<int*>(ck + a.ccap);
+        int* cp = ci + a.ccap;
+        if (!overflow) {
+            for (int p = 0, dst = 0; p < C; dst += end_all[p], ++p)
+                for (int i = tid; i < end_all[p]; i += kThreads) {
+                    ck[dst + i] = ckey[p * cs + i];
+                    ci[dst + i] = cidx[p * cs + i];
+                    cp[dst + i] = cpage[p * cs + i];
+                }
+            __syncthreads();
+        }
+        if (!overflow) {
+            // exact ranks in (key desc, index asc) over the m candidates
+            for (int i = tid; i < m; i += kThreads) {
+                const uint32_t ki = ck[i];
+                const int xi = ci[i];
+                int r0 = 0, r1 = 0;
+                int t = 0;
+                for (; t + 2 <= m; t += 2) {
+                    const uint32_t k0 = ck[t], k1 = ck[t + 1];
+                    r0 += (k0 > ki) | ((k0 == ki) & (ci[t] < xi));
+                    r1 += (k1 > ki) | ((k1 == ki) & (ci[t + 1] < xi));
+                }
+                if (t < m) r0 += (ck[t] > ki) | ((ck[t] == ki) & (ci[t] < xi));
+                crank[i] = r0 + r1;
+            }
+            __syncthreads();
+            for (int i = tid; i < m; i += kThreads) {
+                if (crank[i] >= k) continue;
+                const int xi = ci[i];
+                int p0c = 0, p1c = 0;
+                int t = 0;
+                for (; t + 2 <= m; t += 2) {
+                    p0c += (crank[t] < k) & (ci[t] < xi);
+                    p1c += (crank[t + 1] < k) & (ci[t + 1] < xi);
+                }
+                if (t < m) p0c += (crank[t] < k) & (ci[t] < xi);
+                const int pos = p0c + p1c;
+                sel[pos] = xi;
+                sel_page[pos] = cp[i];
+            }
+        } else {
+            // too many candidates (e.g. many equal scores): gather every score into the idle
+            // ring and run the exact selection there; pages come from the owning CTAs
+            uint32_t* kfull = reinterpret_cast<uint32_t*>(dyn);
+            uint32_t* gscr = kfull + ((NC + 3) & ~3);
+            uint32_t* bkey = gscr + ((NC + 3) / 4 + 4);
+            int* bidx = reinterpret_cast<int*>(bkey + 1024);
+            int* brank = bidx + 1024;
+            for (int j = tid; j < NC; j += kThreads) {
+                const int p = j / slice;
+                kfull[j] = p == r ? keys[j - j0] : ld_peer_u32(peer_addr(keys + (j - p * slice), p));
+            }
+            __syncthreads();
+            select_fast<kThreads>(kfull, NC, NC, k, sel, a.sel_cap, gscr, bkey, bidx, brank, 1024, misc + 2, hist,
+                                  warp_tot, sh);
+            __syncthreads();
+            for (int i = tid; i < k; i += kThreads) {
+                const int j = sel[i];
+                const int p = j / slice;
+                sel_page[i] = p == r ? pages[j - j0] : (int)ld_peer_u32(peer_addr(pages + (j - p * slice), p));
+            }
+        }
+        for (int i = tid; i < L; i += kThreads) {
+            sel[k + i] = NC + i;
+            sel_page[k + i] = i < kMaxLocal ? local_page[i] : -1;
+        }
+    }
+    __syncthreads();
+    if (r == 0) {
+        if (a.sel_idx)
+            for (int i = tid; i < n_sel && i < a.n_max; i += kThreads)
+                a.sel_idx[((int64_t)s * c.H_kv + h) * a.n_max + i] = sel[i];
+        if (a.sel_cnt && tid == 0) a.sel_cnt[s * c.H_kv + h] = min(n_sel, a.n_max);
+    }
+
+    // ---------------- phase 3: decode this CTA's share of the selection ----------------
+    const int i0 = (int)((int64_t)n_sel * r / C), i1 = (int)((int64_t)n_sel * (r + 1) / C);
+    const bool tile_refresh = n_new > 0 && !touched_scored;
+    const int E = G * kHeadDim;         // merge elements (row, channel) of this group
+    const int share = (E + C - 1) / C;  // elements merged by each CTA
+    if (warp == kProducer) {
+        // page ids the selection did not carry (locals past kMaxLocal, or all blocks when
+        // every candidate is taken) are looked up here, 32 at a time
+        for (int g0 = i0; g0 < i1; g0 += 32) {
+            const int i = g0 + lane;
+            if (i < i1 && sel_page[i] < 0) {
+                const int j = sel[i];
+                sel_page[i] = (j >= 0 && j < N) ? (int)page_of(c, s, j, c.status) : -1;
+            }
+        }
+        __syncwarp();
+        bool alive = true;
+        for (int i = i0; i < i1; ++i, ++fill) {
+            const int st = fill % NSt;
+            if (lane == 0 && alive) {
+                if (fill >= (uint32_t)NSt) alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
+                if (alive) {
+                    const int j = sel[i];
+                    const int pg = (j >= 0 && j < N) ? sel_page[i] : -1;
+                    StageInfo inf;
+                    inf.j = j;
+                    inf.valid = pg >= 0 ? min(kBlk, len - j * kBlk) : 0;
+                    inf.ok = pg >= 0;
+                    inf.pos = i;
+                    info[st] = inf;
+                    if (pg >= 0) {
+                        uint8_t* base = dyn + (size_t)st * TG::kStage;
+                        const int y = (pg * c.H_kv + h) * kBlk;
+                        mbar_arrive_expect_tx(&full[st], TG::kStage);
+                        tma_load_2d(base, &tmK, &full[st], 0, y);
+                        tma_load_2d(base + TG::kHalf, &tmK, &full[st], 64, y);
+                        tma_load_2d(base + 2 * TG::kHalf, &tmV, &full[st], 0, y);
+                        tma_load_2d(base + 3 * TG::kHalf, &tmV, &full[st], 64, y);
+                    } else {
+                        report(c.status, SBA_DEV_BAD_SELECTION);
+                        mbar_arrive(&full[st]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    } else {
+        uint32_t qa[8][4];
+        load_q_frags(qa, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
+        const int rr = lane >> 2;
+        const int grp = warp / kGW, gw = warp % kGW;  // consumer group, token slot
+        DecodeState dst;
+        decode_state_init(dst);
+        bool alive = true;
+        for (int i = i0; i < i1; ++i, ++fill) {
+            if ((int)(fill & 1) != grp) continue;  // the other group's block
+            const int st = fill % NSt;
+            if (alive) alive = mbar_wait(&full[st], (fill / NSt) & 1, c.status);
+            const StageInfo inf = info[st];
+            uint8_t* stage = dyn + (size_t)st * TG::kStage;
+            if (inf.ok) {
+                // SAS log-gate of this block (natural log), 0 for the current block B0
+                float b0 = 0.f, b1 = 0.f;
+                if (kScorer == SBA_SCORER_GATE && inf.j != N - 1) {
+                    const int owner = inf.j / slice, off = inf.j - owner * slice;
+                    if (rr < G) b0 = ld_peer_f32(peer_addr(u_s + rr * slice + off, owner)) - lse_s[rr];
+                    if (rr + 8 < G) b1 = ld_peer_f32(peer_addr(u_s + (rr + 8) * slice + off, owner)) - lse_s[rr + 8];
+                }
+                if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && (lane & 3) == 0 && inf.pos < a.n_max) {
+                    if (rr < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr) * a.n_max + inf.pos] = b0;
+                    if (rr + 8 < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr + 8) * a.n_max + inf.pos] = b1;
+                }
+                if (alive)
+                    decode_block<kBlk>(dst, qa, stage, inf.valid, b0 * kLog2e, b1 * kLog2e, a.scale_log2, gw, lane);
+                // (the condition below depends only on the stage info, the same for all four warps)
+                if (tile_refresh && inf.j >= tb0 && inf.j <= tb1) {
+                    // descriptor of a touched (local) block from its staged K tile (the group's
+                    // 128 threads, one channel each)
+                    named_sync(1 + grp, kGW * 32);
+                    const int ch = tid - grp * kGW * 32;
+                    const uint8_t* khalf = stage + (ch >> 6) * TG::kHalf;
+                    const int cc = (ch & 63) >> 3, e = ch & 7;
+                    float lo4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+                    float hi4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    float sm4[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int t0 = 0; t0 < inf.valid; t0 += 4) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int t = t0 + u;
+                            if (t < inf.valid) {
+                                const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                    khalf + t * 128 + ((cc ^ (t & 7)) << 4) + e * 2));
+                                lo4[u] = fminf(lo4[u], x);
+                                hi4[u] = fmaxf(hi4[u], x);
+                                sm4[u] += x;
+                            }
+                        }
+                    }
+                    const float lo = fminf(fminf(lo4[0], lo4[1]), fminf(lo4[2], lo4[3]));
+                    const float hi = fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3]));
+                    const float sum = (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
+                    const int64_t pg = sel_page[inf.pos];
+                    if (kScorer == SBA_SCORER_QUEST) {
+                        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(c.desc) + (pg * c.H_kv + h) * 2 * kHeadDim;
+                        d[ch] = __float2bfloat16_rn(lo);
+                        d[kHeadDim + ch] = __float2bfloat16_rn(hi);
+                    } else {
+                        // pooled summary of the current block, pushed to every CTA for the projection
+                        const float avg = sum / (float)inf.valid;
+                        for (int p = 0; p < C; ++p) {
+                            st_peer_f32(peer_addr(&pooled_b0[ch], p), hi);
+                            st_peer_f32(peer_addr(&pooled_b0[kHeadDim + ch], p), lo);
+                            st_peer_f32(peer_addr(&pooled_b0[2 * kHeadDim + ch], p), avg);
+                        }
+                    }
+                    named_sync(1 + grp, kGW * 32);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        named_sync(3, kCW * 32);  // every consumer is done with the ring before it becomes the merge area
+        decode_state_store(dst, merge_o, merge_ml, warp, lane);
+        named_sync(3, kCW * 32);
+        // this CTA's partial (O, LSE) of every element, pushed to the element's merging CTA
+        for (int e = tid; e < E; e += kCW * 32) {
+            const int row = e / kHeadDim, ch = e % kHeadDim;
+            float o, lse;
+            merge_warps(merge_o, merge_ml, row, ch, o, lse, kCW);
+            const int p = e / share;
+            st_peer_f32(peer_addr(recv_o + r * share + (e - p * share), p), o);
+            if (ch < C) st_peer_f32(peer_addr(&lse_all[r * G + row], ch), lse);
+        }
+    }
+
+    // ---------------- phase 4: merge the cluster's partials (local data only) ----------------
+    cluster_sync();  // every partial pushed; no shared memory is read remotely after this
+    {
+        const int e0 = r * share, e1 = min(e0 + share, E);
+        for (int e = e0 + tid; e < e1; e += kThreads) {
+            const int row = e / kHeadDim, ch = e % kHeadDim;
+            float M = -INFINITY;
+            for (int p = 0; p < C; ++p) M = fmaxf(M, lse_all[p * G + row]);
+            float o = 0.f, W = 0.f;
+            if (M > -INFINITY) {
+                for (int p = 0; p < C; ++p) {
+                    const float l = lse_all[p * G + row];
+                    if (l == -INFINITY) continue;
+                    const float wgt = expf(l - M);
+                    W += wgt;
+                    o = fmaf(wgt, recv_o[p * share + (e - e0)], o);
+                }
+                o /= W;
+            }
+            const int64_t orow = (int64_t)s * c.H_q + h * G + row;
+            if (a.out_dtype == SBA_OUT_BF16)
+                reinterpret_cast<__nv_bfloat16*>(a.out)[orow * kHeadDim + ch] = __float2bfloat16_rn(o);
+            else
+                reinterpret_cast<float*>(a.out)[orow * kHeadDim + ch] = o;
+            if (ch == 0 && a.lse_out) a.lse_out[orow] = W > 0.f ? M + logf(W) : -INFINITY;
+        }
+    }
+    if (kScorer == SBA_SCORER_GATE && tile_refresh && N >= 1 && tb1 == N - 1) {
+        // gate key of the refreshed current block: CTA r computes its channels of kg = A pooled
+        const int c0 = kHeadDim * r / C, c1 = kHeadDim * (r + 1) / C;
+        const int pg = page_quiet(c, s, N - 1);
+        for (int ch = c0 + warp; ch < c1; ch += kThreads / 32) {
+            const float* Ar = a.gate_A + (int64_t)ch * 3 * kHeadDim;
+            float acc = 0.f;
+            for (int i = lane; i < 3 * kHeadDim; i += 32) acc = fmaf(__ldg(Ar + i), pooled_b0[i], acc);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0 && pg >= 0) c.kg[((int64_t)pg * c.H_kv + h) * kHeadDim + ch] = acc;
+        }
+    }
+}
+
+// A = Wq^T Wk / sqrt(dg): the gate projection folded into query space.
+__global__ void fold_gate_kernel(const float* __restrict__ Wq, const float* __restrict__ Wk, int dg, float* A) {
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // over 128 x 384
+    if (idx >= kHeadDim * 3 * kHeadDim) return;
+    const int ch = idx / (3 * kHeadDim), i = idx % (3 * kHeadDim);
+    float acc = 0.f;
+    for (int r = 0; r < dg; ++r) acc = fmaf(__ldg(Wq + (int64_t)r * kHeadDim + ch), __ldg(Wk + (int64_t)r * 3 * kHeadDim + i), acc);
+    A[idx] = acc * rsqrtf((float)dg);
+}
+
+struct Plan {
+    int C, n_stages, smem, slice, gcap, ccap, sel_cap;
+    int off_keys, off_pages, off_u, off_gmax, off_ckey, off_cidx, off_cpage, off_crank, off_sel, off_selp, off_recv,
+        off_bars;
+};
+
+int round4(int x) { return (x + 3) & ~3; }
+
+Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_sel) {
+    Plan pl{};
+    pl.C = C;
+    const int G = c.H_q / c.H_kv;
+    const int stage = c.b * kDescBytes;
+    pl.slice = round4((c.max_blocks + C - 1) / C);
+    pl.gcap = round4((pl.slice + 3) / 4);
+    pl.ccap = 1024;
+    pl.sel_cap = round4(n_max_sel);
+    const int E = G * kHeadDim;
+    int off = 0;
+    auto take = [&](int words) {
+        const int o = off;
+        off += round4(words) * 4;
+        return o;
+    };
+    // the ring comes first (1024-aligned); the fallback selection reuses it
+    const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + (c.b == 64 ? 1 : 0);
+    int ns = 6;
+    const int fixed_bytes = 4 * (round4(pl.slice) * 2 + (p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0) +
+                                 C * pl.gcap + 4 * pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
+    const int budget = 227 * 1024 - 1024 /*align*/ - 8 * 1024 /*static shared memory headroom*/;
+    while (ns > max(2, min_stages) && ns * stage + fixed_bytes + ns * (16 + (int)sizeof(StageInfo)) > budget) --ns;
+    pl.n_stages = ns;
+    off = ns * stage;
+    pl.off_keys = take(pl.slice);
+    pl.off_pages = take(pl.slice);
+    pl.off_u = take(p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0);
+    pl.off_gmax = take(C * pl.gcap);
+    pl.off_ckey = take(pl.ccap);
+    pl.off_cidx = take(pl.ccap);
+    pl.off_cpage = take(pl.ccap);
+    pl.off_crank = take(pl.ccap);
+    pl.off_sel = take(pl.sel_cap);
+    pl.off_selp = take(pl.sel_cap);
+    pl.off_recv = take(C * ((E + C - 1) / C));
+    pl.off_bars = off;
+    pl.smem = pl.off_bars + ns * (16 + (int)sizeof(StageInfo)) + 1024;
+    // the fallback selection needs max_blocks + max_blocks/4 + 3*1024 words of the ring
+    if ((c.max_blocks + c.max_blocks / 4 + 8 + 3 * 1024) * 4 > ns * stage) pl.smem = 1 << 30;
+    return pl;
+}
+
+template <int kBlk, int kScorer, int kGM>
+cudaError_t prepare_kernel(int smem) {
+    auto kern = decode_step_kernel<kBlk, kScorer, kGM>;
+    if (allow_smem<decode_step_kernel<kBlk, kScorer, kGM>>(smem) != SBA_OK) return cudaErrorInvalidValue;
+    static bool nonportable_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !nonportable_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        nonportable_set[dev] = true;
+    }
+    return cudaSuccess;
+}
+
+cudaLaunchConfig_t step_config(const sba_cache& c, const Plan& pl, cudaStream_t stream, cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.C, c.H_kv, c.B);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    return cfg;
+}
+
+// Clusters of this size the device can keep resident at once (0 if none).
+template <int kBlk, int kScorer, int kGM>
+int active_clusters(const sba_cache& c, const Plan& pl) {
+    if (prepare_kernel<kBlk, kScorer, kGM>(pl.smem) != cudaSuccess) return 0;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = step_config(c, pl, nullptr, attr);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, decode_step_kernel<kBlk, kScorer, kGM>, &cfg) != cudaSuccess) return 0;
+    return active;
+}
+
+// Kernel instantiation for a cache shape: block size, scorer, and (gate) the
+// head count rounded up to a power of two.
+template <class F>
+int dispatch(const sba_cache& c, const sba_select_params& p, F&& f) {
+    const int G = c.H_q / c.H_kv;
+    if (p.scorer == SBA_SCORER_QUEST)
+        return c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1>() : f.template run<128, SBA_SCORER_QUEST, 1>();
+    if (G <= 4) return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 4>() : f.template run<128, SBA_SCORER_GATE, 4>();
+    if (G <= 8) return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 8>() : f.template run<128, SBA_SCORER_GATE, 8>();
+    return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 16>() : f.template run<128, SBA_SCORER_GATE, 16>();
+}
+
+struct ActiveClusters {
+    const sba_cache& c;
+    const Plan& pl;
+    template <int kBlk, int kScorer, int kGM>
+    int run() {
+        return active_clusters<kBlk, kScorer, kGM>(c, pl);
+    }
+};
+
+int active_clusters_any(const sba_cache& c, const sba_select_params& p, const Plan& pl) {
+    return dispatch(c, p, ActiveClusters{c, pl});
+}
+
+template <int kBlk, int kScorer, int kGM>
+int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaStream_t stream) {
+    CUtensorMap tk, tv;
+    const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
+    if (!make_kv_tmap(&tk, c.k, rows, kBlk) || !make_kv_tmap(&tv, c.v, rows, kBlk)) return SBA_ERR_CUDA;
+    cudaError_t e = prepare_kernel<kBlk, kScorer, kGM>(pl.smem);
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return SBA_ERR_CUDA;
+    }
+    StepArgs a = a0;
+    a.n_stages = pl.n_stages;
+    a.slice = pl.slice;
+    a.off_keys = pl.off_keys;
+    a.off_pages = pl.off_pages;
+    a.off_u = pl.off_u;
+    a.off_gmax = pl.off_gmax;
+    a.off_ckey = pl.off_ckey;
+    a.off_cidx = pl.off_cidx;
+    a.off_cpage = pl.off_cpage;
+    a.off_crank = pl.off_crank;
+    a.off_sel = pl.off_sel;
+    a.off_selp = pl.off_selp;
+    a.off_recv = pl.off_recv;
+    a.off_bars = pl.off_bars;
+    a.gcap = pl.gcap;
+    a.ccap = pl.ccap;
+    a.sel_cap = pl.sel_cap;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = step_config(c, pl, stream, attr);
+    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM>, tk, tv, a);
+    if (e != cudaSuccess) {
+        note_cuda_error(e);
+        return SBA_ERR_CUDA;
+    }
+    return SBA_OK;
+}
+
+struct LaunchStep {
+    const sba_cache& c;
+    const StepArgs& a;
+    const Plan& pl;
+    cudaStream_t stream;
+    template <int kBlk, int kScorer, int kGM>
+    int run() {
+        return launch_step_t<kBlk, kScorer, kGM>(c, a, pl, stream);
+    }
+};
+
+int n_max_selected(const sba_cache& c, const sba_select_params& p) {
+    const int N_max = (c.max_len + c.b - 1) / c.b;
+    return num_selected(N_max, p) > 0 ? num_selected(N_max, p) : 1;
+}
+
+}  // namespace
+
+int step_cluster_size(const sba_cache& c, const sba_select_params& p, int num_sms) {
+    // one CTA per SM: the largest C <= 16 with B*H_kv*C <= #SMs whose clusters are all
+    // resident at once; failing that, the largest schedulable C
+    const int64_t units = (int64_t)c.B * c.H_kv;
+    int start = kMaxCluster;
+    while (start > 1 && units * start > num_sms) --start;
+    for (int pass = 0; pass < 2; ++pass)
+        for (int C = start; C >= 1; --C) {
+            const Plan pl = plan_step(c, p, C, n_max_selected(c, p));
+            if (pl.smem > 227 * 1024) return 0;
+            const int active = active_clusters_any(c, p, pl);
+            if (active >= 1 && (pass == 1 || C == 1 || active >= units)) return C;
+        }
+    return 0;
+}
+
+int launch_decode_step(const sba_cache& c, const void* q, const void* k_new, const void* v_new,
+                       const int32_t* pos_start, int n_new, const float* gate_A, const sba_select_params& p,
+                       float scale, void* out, int out_dtype, float* lse_out, int32_t* sel_idx, int32_t* sel_cnt,
+                       float* gate_bias, int n_max, int cluster, cudaStream_t stream) {
+    if (cluster < 1) return SBA_ERR_UNSUPPORTED;
+    const Plan pl = plan_step(c, p, cluster, n_max_selected(c, p));
+    if (pl.smem > 227 * 1024) return SBA_ERR_UNSUPPORTED;
+    StepArgs a{};
+    a.c = c;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.k_new = reinterpret_cast<const uint4*>(k_new);
+    a.v_new = reinterpret_cast<const uint4*>(v_new);
+    a.pos_start = pos_start;
+    a.n_new = n_new;
+    a.gate_A = gate_A;
+    a.p = p;
+    a.scale_log2 = scale * kLog2e;
+    a.out = out;
+    a.out_dtype = out_dtype;
+    a.lse_out = lse_out;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.gate_bias = gate_bias;
+    a.n_max = n_max;
+    return dispatch(c, p, LaunchStep{c, a, pl, stream});
+}
+
+int launch_fold_gate(const float* Wq, const float* Wk, int dg, float* A, cudaStream_t stream) {
+    const int n = kHeadDim * 3 * kHeadDim;
+    return launch(fold_gate_kernel, dim3((n + 255) / 256), dim3(256), 0, stream, Wq, Wk, dg, A);
+}
+
+}  // namespace sba

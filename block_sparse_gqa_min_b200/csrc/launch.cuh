@@ -77,6 +77,12 @@ int launch_score_select(const sba_cache& c, const void* q, const sba_select_para
 int launch_sparse_decode(const sba_cache& c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
                          const float* gate_bias, int n_max, float scale, int num_splits, float* o_part,
                          float* lse_part, cudaStream_t stream);
+int step_cluster_size(const sba_cache& c, const sba_select_params& p, int num_sms);
+int launch_decode_step(const sba_cache& c, const void* q, const void* k_new, const void* v_new,
+                       const int32_t* pos_start, int n_new, const float* gate_A, const sba_select_params& p,
+                       float scale, void* out, int out_dtype, float* lse_out, int32_t* sel_idx, int32_t* sel_cnt,
+                       float* gate_bias, int n_max, int cluster, cudaStream_t stream);
+int launch_fold_gate(const float* Wq, const float* Wk, int dg, float* A, cudaStream_t stream);
 int launch_combine(const float* o_part, const float* lse_part, int B, int H_q, int S, void* out, int out_dtype,
                    float* lse_out, cudaStream_t stream);
 

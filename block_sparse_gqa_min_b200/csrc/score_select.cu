@@ -23,6 +23,7 @@
 
 #include "common.cuh"
 #include "launch.cuh"
+#include "select.cuh"
 
 namespace sba {
 
@@ -32,6 +33,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBlocksPerWarpIter = 8;  // 4 lanes per block descriptor (512 B)
 constexpr int kRefSMs = 148;
+constexpr int kSelCap = 1024;  // selection buffer (candidates above the group-maximum bound)
 
 struct ScoreArgs {
     sba_cache c;
@@ -68,124 +70,6 @@ WsLayout ws_layout(const sba_cache& c, const sba_select_params& p, int chunk) {
     return w;
 }
 
-// Exclusive prefix over the 8 warps of per-warp totals held in smem.
-__device__ __forceinline__ int warp_prefix(const int* warp_tot, int warp) {
-    int acc = 0;
-    for (int w = 0; w < warp; ++w) acc += warp_tot[w];
-    return acc;
-}
-
-// ---------------------------------------------------------------------------
-// Selection over NC ranked candidates (keys in smem) plus the forced local
-// blocks [NC, N).  Writes ascending indices to out[0..min(n_sel, n_max)).
-// k = number of candidates to take.  Runs on all 256 threads.
-// ---------------------------------------------------------------------------
-__device__ void select_and_compact(const uint32_t* keys, int NC, int N, int k, int32_t* out, int n_max,
-                                   uint32_t* hist, int* warp_tot, uint32_t* sh) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // mode: 0 = threshold (0 < k < NC), 1 = take all candidates, 2 = take none
-    const int mode = k >= NC ? 1 : (k <= 0 ? 2 : 0);
-    uint32_t T = 0;
-    int rem = 0;
-    if (mode == 0) {
-        uint32_t prefix = 0, pmask = 0;
-        rem = k;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            hist[tid] = 0;
-            __syncthreads();
-            for (int j = tid; j < NC; j += kThreads) {
-                const uint32_t kk = keys[j];
-                if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & 255u], 1u);
-            }
-            __syncthreads();
-            if (warp == 0) {
-                uint32_t cnt[8], lsum = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    cnt[e] = hist[255 - 8 * lane - e];
-                    lsum += cnt[e];
-                }
-                uint32_t incl = lsum;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += t;
-                }
-                const uint32_t excl = incl - lsum;
-                if (excl < (uint32_t)rem && (uint32_t)rem <= incl) {
-                    uint32_t run = excl;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        if (run + cnt[e] >= (uint32_t)rem) {
-                            sh[0] = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
-                            sh[1] = (uint32_t)rem - run;
-                            break;
-                        }
-                        run += cnt[e];
-                    }
-                }
-            }
-            __syncthreads();
-            prefix = sh[0];
-            rem = (int)sh[1];
-            pmask |= 0xffu << shift;
-        }
-        T = prefix;  // exact key of the n-th candidate; `rem` equal keys are taken, lowest index first
-    }
-    // Per-warp contiguous segments, processed 32 consecutive indices at a time,
-    // so that ranks among equal keys and output positions follow index order.
-    const int seg = ((N + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-    const int jb = warp * seg, je = min(N, jb + seg);
-    const unsigned lt = (1u << lane) - 1u;
-    // pass A: ties per warp
-    int eq_w = 0;
-    if (mode == 0)
-        for (int base = jb; base < je; base += 32) {
-            const int j = base + lane;
-            const bool is_eq = j < je && j < NC && keys[j] == T;
-            eq_w += __popc(__ballot_sync(0xffffffffu, is_eq));
-        }
-    if (lane == 0) warp_tot[warp] = eq_w;
-    __syncthreads();
-    const int eq_before = warp_prefix(warp_tot, warp);
-    __syncthreads();
-    // pass B: selected per warp; pass C: write
-    for (int pass = 0; pass < 2; ++pass) {
-        int er = eq_before, sel_run = 0;
-        int out_base = 0;
-        if (pass == 1) out_base = warp_prefix(warp_tot, warp);
-        for (int base = jb; base < je; base += 32) {
-            const int j = base + lane;
-            bool sel = false, is_eq = false;
-            if (j < je) {
-                if (j >= NC) {
-                    sel = true;
-                } else if (mode == 1) {
-                    sel = true;
-                } else if (mode == 0) {
-                    const uint32_t kk = keys[j];
-                    is_eq = kk == T;
-                    sel = kk > T;
-                }
-            }
-            const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-            if (is_eq) sel = (er + __popc(eqm & lt)) < rem;
-            er += __popc(eqm);
-            const unsigned sm = __ballot_sync(0xffffffffu, sel);
-            if (pass == 1 && sel) {
-                const int pos = out_base + sel_run + __popc(sm & lt);
-                if (pos < n_max) out[pos] = j;
-            }
-            sel_run += __popc(sm);
-        }
-        if (pass == 0) {
-            __syncthreads();
-            if (lane == 0) warp_tot[warp] = sel_run;
-            __syncthreads();
-        }
-    }
-}
-
 template <int kScorer>
 __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
     extern __shared__ __align__(16) uint8_t dyn[];
@@ -193,6 +77,7 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
     __shared__ int warp_tot[kWarps];
     __shared__ uint32_t sh[2];
     __shared__ int is_last;
+    __shared__ int sel_misc[2];
     __shared__ float lse_s[kMaxGroup];
     __shared__ __align__(16) float q_s[kMaxGroup][kHeadDim];
 
@@ -392,7 +277,14 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
     }
     __syncthreads();
     int32_t* out = a.sel_idx + ((int64_t)s * c.H_kv + h) * a.n_max;
-    select_and_compact(keys, NC, N, k, out, a.n_max, hist, warp_tot, sh);
+    {
+        uint32_t* gscr = reinterpret_cast<uint32_t*>(dyn + (main_words + a.chunk) * 4);
+        uint32_t* bkey = gscr + (mb + 3) / 4 + 4;
+        int* bidx = reinterpret_cast<int*>(bkey + kSelCap);
+        int* brank = bidx + kSelCap;
+        select_fast<kThreads>(keys, NC, N, k, out, a.n_max, gscr, bkey, bidx, brank, kSelCap, sel_misc, hist, warp_tot,
+                              sh);
+    }
     if (n_sel > a.n_max && tid == 0) report(c.status, SBA_DEV_BAD_SELECTION);
     const int n_out = min(n_sel, a.n_max);
     if (tid == 0) a.sel_cnt[s * c.H_kv + h] = n_out;
@@ -425,7 +317,8 @@ size_t score_workspace_bytes(const sba_cache& c, const sba_select_params& p) {
 static size_t score_smem_bytes(const sba_cache& c, int chunk) {
     const int G = c.H_q / c.H_kv;
     const size_t main_words = c.max_blocks > G * chunk ? (size_t)c.max_blocks : (size_t)G * chunk;
-    return main_words * 4 + (size_t)chunk * 4;
+    const size_t sel_words = (size_t)(c.max_blocks + 3) / 4 + 4 + 3 * kSelCap;
+    return (main_words + chunk + sel_words) * 4;
 }
 
 int launch_score_select(const sba_cache& c, const void* q, const sba_select_params& p, int32_t* sel_idx,

@@ -93,6 +93,10 @@ _SIGS = {
     "sba_sparse_decode": ([ctypes.POINTER(sba_cache), _P, _P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _P],
                           ctypes.c_int),
     "sba_combine": ([_P, _P, _I, _I, _I, _I, _P, _I, _P, _P], ctypes.c_int),
+    "sba_fold_gate": ([ctypes.POINTER(sba_gate), _P, _P], ctypes.c_int),
+    "sba_decode_step_cluster": ([ctypes.POINTER(sba_cache), ctypes.POINTER(sba_select_params)], _I),
+    "sba_decode_step": ([ctypes.POINTER(sba_cache), _P, _P, _P, _P, _I, _P, ctypes.POINTER(sba_select_params),
+                         ctypes.c_float, _P, _I, _P, _P, _P, _P, _I, _P], ctypes.c_int),
 }
 
 _lib = None
@@ -245,6 +249,31 @@ def sba_combine(o_part: torch.Tensor, lse_part: torch.Tensor, out: torch.Tensor,
         raise ValueError("out must be fp32 or bf16")
     _check(load().sba_combine(_ptr(o_part), _ptr(lse_part), B, H_q, S, d, _ptr(out), dt, _ptr(lse_out),
                               _stream(stream)), "sba_combine")
+
+
+def sba_fold_gate(Wq: torch.Tensor, Wk: torch.Tensor, A: torch.Tensor, stream=None):
+    _check(load().sba_fold_gate(ctypes.byref(sba_gate(_ptr(Wq), _ptr(Wk), int(Wq.shape[0]))), _ptr(A),
+                                _stream(stream)), "sba_fold_gate")
+
+
+def sba_decode_step_cluster(c: Cache, p: sba_select_params) -> int:
+    return int(load().sba_decode_step_cluster(ctypes.byref(c.struct()), ctypes.byref(p)))
+
+
+def sba_decode_step(c: Cache, q: torch.Tensor, p: sba_select_params, softmax_scale: float, out: torch.Tensor,
+                    lse_out: Optional[torch.Tensor] = None, k_new: Optional[torch.Tensor] = None,
+                    v_new: Optional[torch.Tensor] = None, pos_start: Optional[torch.Tensor] = None,
+                    gate_A: Optional[torch.Tensor] = None, sel_idx: Optional[torch.Tensor] = None,
+                    sel_cnt: Optional[torch.Tensor] = None, gate_bias: Optional[torch.Tensor] = None,
+                    stream=None):
+    n_new = 0 if k_new is None else int(k_new.shape[1])
+    n_max = int(sel_idx.shape[-1]) if sel_idx is not None else (int(gate_bias.shape[-1]) if gate_bias is not None
+                                                               else 0)
+    dt = SBA_OUT_BF16 if out.dtype == torch.bfloat16 else SBA_OUT_F32
+    _check(load().sba_decode_step(ctypes.byref(c.struct()), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(pos_start),
+                                  n_new, _ptr(gate_A), ctypes.byref(p), float(softmax_scale), _ptr(out), dt,
+                                  _ptr(lse_out), _ptr(sel_idx), _ptr(sel_cnt), _ptr(gate_bias), n_max,
+                                  _stream(stream)), "sba_decode_step")
 
 
 # ---------------------------------------------------------------------------

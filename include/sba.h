@@ -232,6 +232,43 @@ int sba_combine(const float *o_part, const float *lse_part, int32_t B, int32_t H
                 int32_t num_splits, int32_t d, void *out, int32_t out_dtype, float *lse_out,
                 void *stream);
 
+/* Fold the gate projection into query space once per layer:
+ * A = Wq^T Wk / sqrt(dg), device fp32 [d][3d] (row-major), so that the stored
+ * gate key of a block is kg = A pooled and its gate logit for a query head is
+ * u = q . kg ("SAS ...", Method; "SeerAttention-R ...", abstract).  Used by
+ * sba_decode_step. */
+int sba_fold_gate(const sba_gate *gate, float *A, void *stream);
+
+/* Cluster size (CTAs per sequence and KV group) that sba_decode_step uses on
+ * the current device for this cache shape and rule: the largest power of two
+ * <= 16 with every cluster resident at once when possible (one CTA per SM).
+ * Sets kernel attributes, launches nothing; 0 if the shape is not supported
+ * by the fused step. */
+int32_t sba_decode_step_cluster(const sba_cache *c, const sba_select_params *p);
+
+/* One whole decode step of one layer in ONE launch: rows a1-a6 fused.
+ * 1. append n_new tokens per sequence at pos_start[s] (as sba_append_kv;
+ *    n_new = 0 skips steps 1-2, pos_start may then be NULL);
+ * 2. recompute the descriptors of the blocks those tokens touch (as
+ *    sba_update_descriptors; the gate path uses the folded gate_A);
+ * 3-4. score and select exactly as sba_score_select;
+ * 5-6. attention over the selected blocks and the merge, as sba_sparse_decode
+ *    followed by sba_combine, writing out [B][H_q][d] (SBA_OUT_F32 or
+ *    SBA_OUT_BF16) and lse_out [B][H_q] (fp32, may be NULL).
+ * sel_idx/sel_cnt/gate_bias (layouts of sba_score_select, each may be NULL)
+ * report the selection; n_max is their row length.
+ * The caller advances seq_lens to include the appended tokens BEFORE the call.
+ * Each (sequence, KV head) runs on one thread-block cluster of up to 16 CTAs
+ * (one per SM); scores, the selection and the partial outputs stay in (shared
+ * and distributed shared) memory, so the call needs no workspace.  A step whose
+ * appended tokens touch a block it also scores (e.g. n_local = 0) refreshes
+ * that block before scoring, at the cost of one extra cluster barrier. */
+int sba_decode_step(const sba_cache *c, const void *q, const void *k_new, const void *v_new,
+                    const int32_t *pos_start, int32_t n_new, const float *gate_A,
+                    const sba_select_params *p, float softmax_scale, void *out, int32_t out_dtype,
+                    float *lse_out, int32_t *sel_idx, int32_t *sel_cnt, float *gate_bias, int32_t n_max,
+                    void *stream);
+
 #ifdef __cplusplus
 }
 #endif
