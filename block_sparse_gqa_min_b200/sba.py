@@ -94,6 +94,9 @@ _SIGS = {
                           ctypes.c_int),
     "sba_combine": ([_P, _P, _I, _I, _I, _I, _P, _I, _P, _P], ctypes.c_int),
     "sba_fold_gate": ([ctypes.POINTER(sba_gate), _P, _P], ctypes.c_int),
+    "sba_static_scratch_bytes": ([], ctypes.c_size_t),
+    "sba_score_select_static": ([ctypes.POINTER(sba_cache), _P, ctypes.POINTER(sba_select_params), _P, _P, _P, _I,
+                                 _P], ctypes.c_int),
     "sba_decode_step_cluster": ([ctypes.POINTER(sba_cache), ctypes.POINTER(sba_select_params)], _I),
     "sba_decode_step": ([ctypes.POINTER(sba_cache), _P, _P, _P, _P, _I, _P, ctypes.POINTER(sba_select_params),
                          ctypes.c_float, _P, _I, _P, _P, _P, _P, _I, _P], ctypes.c_int),
@@ -229,6 +232,20 @@ def sba_score_select(c: Cache, q: torch.Tensor, p: sba_select_params, sel_idx: t
     _check(load().sba_score_select(ctypes.byref(c.struct()), _ptr(q), ctypes.byref(p), _ptr(sel_idx),
                                    _ptr(sel_cnt), _ptr(gate_bias), n_max, _ptr(ws), ws.numel() * ws.element_size(),
                                    _stream(stream)), "sba_score_select")
+
+
+def sba_static_scratch_bytes() -> int:
+    return int(load().sba_static_scratch_bytes())
+
+
+def sba_score_select_static(c: Cache, q: torch.Tensor, p: sba_select_params, sel_idx: torch.Tensor,
+                            sel_cnt: torch.Tensor, gate_bias: Optional[torch.Tensor], stream=None):
+    """sba_score_select without a workspace (for callers that cannot allocate):
+    the library's static per-device scratch is used instead."""
+    n_max = int(sel_idx.shape[-1])
+    _check(load().sba_score_select_static(ctypes.byref(c.struct()), _ptr(q), ctypes.byref(p), _ptr(sel_idx),
+                                          _ptr(sel_cnt), _ptr(gate_bias), n_max, _stream(stream)),
+           "sba_score_select_static")
 
 
 def sba_sparse_decode(c: Cache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,

@@ -232,6 +232,30 @@ int sba_combine(const float *o_part, const float *lse_part, int32_t B, int32_t H
                 int32_t num_splits, int32_t d, void *out, int32_t out_dtype, float *lse_out,
                 void *stream);
 
+/* Size in bytes of the static scratch behind sba_score_select_static (8 MiB). */
+size_t sba_static_scratch_bytes(void);
+
+/* sba_score_select for callers that cannot allocate device memory when they
+ * issue a step: an engine that records its step into a CUDA graph and forbids
+ * cudaMalloc during capture, a serving-framework plugin whose enqueue callback
+ * must not allocate, an embedded runtime with a device-memory budget fixed at
+ * start-up.  No counterpart on the pages: it is a deployment convenience.
+ * Same arguments, semantics and outputs as sba_score_select, without ws and
+ * ws_bytes: the scratch is one static device array of
+ * sba_static_scratch_bytes() bytes that the library reserves on every GPU that
+ * loads it, until the process exits.
+ *  - A problem needing more scratch than that (sba_workspace_size) returns
+ *    SBA_ERR_WORKSPACE before anything is enqueued.
+ *  - The first call on a device looks the array's address up for that device;
+ *    make it before any stream capture.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents; each call first clears the completion counters on `stream`
+ *    (cudaMemsetAsync).  Calls whose kernels can overlap on the GPU (streams
+ *    with no ordering between them) race on the array.
+ *  - Calls no allocating routine (cudaMalloc, cudaFree, library allocators). */
+int sba_score_select_static(const sba_cache *c, const void *q, const sba_select_params *p, int32_t *sel_idx,
+                            int32_t *sel_cnt, float *gate_bias, int32_t n_max, void *stream);
+
 /* Fold the gate projection into query space once per layer:
  * A = Wq^T Wk / sqrt(dg), device fp32 [d][3d] (row-major), so that the stored
  * gate key of a block is kg = A pooled and its gate logit for a query head is
