@@ -91,6 +91,43 @@ def peaks():
         return 6650.0, "fallback"
 
 
+# sources of the fused step kernel: a recorded ncu traffic figure is valid only while they are unchanged
+KERNEL_SOURCES = {
+    "decode_step": ["fused_step.cu", "decode_tile.cuh", "select.cuh", "common.cuh", "launch.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(ROOT, "block_sparse_gqa_min_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) from the committed ncu summary of this
+    kernel and workload, or None when there is none or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != kernel_source_hash(kernel):
+        return None
+    try:
+        return int(float(fields["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
 def counted_bytes(w, seq_lens, n_sel_of):
     """Counted bytes of one layer for the given lengths."""
     tot = 0
@@ -345,7 +382,7 @@ def native(args, rank, world, local):
     roof = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
             "alg_bytes_per_launch": alg[dom], "launch_us": round(kmean[dom] * 1e3, 3),
-            "traffic": None,
+            "traffic": recorded_traffic(dom, w.name),
             "other_kernels_us": {k: round(v * 1e3, 3) for k, v in kmean.items() if k != dom},
             "step_frac": round(step_bytes / (ms_max * 1e-3) / 1e9 / hbm, 4)}
 
