@@ -151,14 +151,27 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
-// 1-D bulk copy (TMA engine) global -> this CTA's shared memory, completing on
-// `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(smem_dst)),
-        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
+// 16-byte asynchronous copy global -> this CTA's shared memory (cached in L2
+// only).  Both addresses 16-byte aligned.  Many small scattered copies go
+// through the load/store unit at full rate, unlike one bulk copy each.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+
+// Make `bar` track this thread's earlier cp.async copies: its pending count is
+// raised now and lowered when they have landed, so the phase cannot complete
+// before them (this is not an arrival of its own).
+__device__ __forceinline__ void cp_async_mbar_track(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 16-byte global load that does not allocate in L1 (data read once per step).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 v;
+    asm("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
 }
 
 // Generic-proxy global writes made visible to later async-proxy (TMA) reads.

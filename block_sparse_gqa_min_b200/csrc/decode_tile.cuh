@@ -173,19 +173,24 @@ __device__ __forceinline__ void decode_block(DecodeState& st, const uint32_t (&q
 }
 
 // This warp's (max, sum, O) rows to shared memory: merge_o [warps][16][128],
-// merge_ml [warps][16][2].
+// merge_ml [warps][16][2].  Rows >= rows_used (zero query rows) are not stored.
 __device__ __forceinline__ void decode_state_store(DecodeState& st, float* merge_o, float* merge_ml, int warp,
-                                                   int lane) {
+                                                   int lane, int rows_used = 16) {
     const int r = lane >> 2, cq = (lane & 3) * 2;
     st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, 1);
     st.l0 += __shfl_xor_sync(0xffffffffu, st.l0, 2);
     st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, 1);
     st.l1 += __shfl_xor_sync(0xffffffffu, st.l1, 2);
     float* mo = merge_o + warp * 16 * kHeadDim;
+    if (r < rows_used) {
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        *reinterpret_cast<float2*>(mo + r * kHeadDim + n * 8 + cq) = make_float2(st.o[n][0], st.o[n][1]);
-        *reinterpret_cast<float2*>(mo + (r + 8) * kHeadDim + n * 8 + cq) = make_float2(st.o[n][2], st.o[n][3]);
+        for (int n = 0; n < 16; ++n)
+            *reinterpret_cast<float2*>(mo + r * kHeadDim + n * 8 + cq) = make_float2(st.o[n][0], st.o[n][1]);
+    }
+    if (r + 8 < rows_used) {
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+            *reinterpret_cast<float2*>(mo + (r + 8) * kHeadDim + n * 8 + cq) = make_float2(st.o[n][2], st.o[n][3]);
     }
     if ((lane & 3) == 0) {
         merge_ml[(warp * 16 + r) * 2] = st.m0;

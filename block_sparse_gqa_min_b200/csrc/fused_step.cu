@@ -5,10 +5,11 @@
 // Efficient Long-Sequence Generation", Summary and Key points; "SAS: Simple
 // Attention Sparsification ...", Method), organised for B200:
 //  - one thread-block CLUSTER of C CTAs (one CTA per SM) per (sequence, KV
-//    group); CTA r owns slice r of the blocks [0, max_blocks) for scoring and
-//    share r of the selected blocks for attention;
-//  - descriptors stream into a shared-memory ring with 1-D bulk copies (TMA
-//    engine, mbarrier completion); K/V tiles with 2-D TMA loads (128-B swizzle);
+//    group); CTA r owns slice r of the sequence's scored blocks and share r
+//    of the selected blocks for attention;
+//  - descriptors stream into a shared-memory ring as 16-byte cp.async gathers
+//    (one warp-wide instruction per 512-byte descriptor, completion tracked by
+//    the stage's mbarrier); K/V tiles with 2-D TMA loads (128-B swizzle);
 //  - the selection is distributed: each CTA pushes the maxima of groups of its
 //    scores to its peers (distributed shared memory); every CTA derives the same
 //    lower bound T0 of the n-th score from them (k group maxima are k distinct
@@ -47,6 +48,7 @@ constexpr int kThreads = (kCW + 1) * 32;
 constexpr int kProducer = kCW;
 constexpr int kMaxCluster = 16;
 constexpr int kDescBytes = 512;
+static_assert(kCW == 8, "the merge weights are read as two float4 per row");
 
 struct StepArgs {
     sba_cache c;
@@ -67,7 +69,7 @@ struct StepArgs {
     int n_max;
     // shared-memory layout (bytes from the 1024-aligned base) and capacities
     int n_stages;
-    int slice;      // blocks of [0, max_blocks) per CTA (multiple of 4)
+    int slice;      // largest slice: ceil(max_blocks / C) rounded up to a multiple of 4
     int off_keys, off_pages, off_u, off_gmax, off_ckey, off_cidx, off_cpage, off_crank, off_sel, off_selp,
         off_recv, off_bars;
     int gcap;       // group maxima per CTA slot
@@ -181,17 +183,17 @@ template <int kBlk, int kScorer, int kGM>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, StepArgs a) {
     using TG = TileGeom<kBlk>;
-    constexpr int kChunk = 64;  // descriptors per ring fill; consecutive fills alternate consumer groups
     constexpr int kMaxLocal = 64;
     __shared__ uint32_t hist[256];
     __shared__ int warp_tot[kThreads / 32];
     __shared__ uint32_t sh[2];
     __shared__ int misc[4];
     __shared__ float lse_s[kMaxGroup];
+    __shared__ __align__(16) float wgt_s[kMaxGroup][kCW];  // merge weights of the consumer warps
     __shared__ float lse_all[kMaxCluster * kMaxGroup];
     __shared__ float mz_all[kMaxCluster * kMaxGroup][2];
-    __shared__ int cnt_g[kMaxCluster];    // group maxima pushed by each CTA
-    __shared__ int end_all[kMaxCluster];  // candidates each CTA pushed
+    __shared__ int end_all[kMaxCluster];    // candidates each CTA pushed
+    __shared__ int pre_s[kMaxCluster + 1];  // their prefix
     __shared__ int local_page[kMaxLocal];
     __shared__ __align__(16) float pooled[3 * kHeadDim];     // refresh-before-score scratch
     __shared__ __align__(16) float pooled_b0[3 * kHeadDim];  // pushed pooled summary of B0
@@ -223,8 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = blockIdx.y, s = blockIdx.z;
     const int G = c.H_q / c.H_kv;
     const int mb = c.max_blocks;
-    const int slice = a.slice;
-    const int j0 = min(r * slice, mb), j1 = min(j0 + slice, mb);
+    const int ustride = a.slice;  // row stride of u_s: the largest slice
 
     if (tid == 0) {
         for (int i = 0; i < NSt; ++i) {
@@ -244,8 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- shapes of this (sequence, group) ----------------
     const int len = __ldg(c.seq_lens + s);
     const int p0raw = a.n_new > 0 ? __ldg(a.pos_start + s) : 0;
-    if (warp == kProducer)  // speculative page ids of the slice while the lengths arrive
-        for (int j = j0 + lane; j < j1; j += 32) pages[j - j0] = page_quiet(c, s, j);
     int N = blocks_of(len, kBlk);
     if (N > mb) {
         if (tid == 0 && r == 0) report(c.status, SBA_DEV_BAD_POSITION);
@@ -255,8 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_sel = min(num_selected(N, a.p), a.sel_cap);
     const int NC = N - L;                                               // ranked candidates [0, NC)
     const int NSc = kScorer == SBA_SCORER_GATE ? max(N - 1, 0) : NC;   // blocks this step scores
-    const int js1 = max(j0, min(j1, NSc));                              // my scored blocks [j0, js1)
-    const int jc1 = max(j0, min(j1, NC));                               // my ranked candidates [j0, jc1)
+    // this sequence's scored blocks [0, NSc) in C equal slices (sequences differ in length)
+    const int slice = min(max(4, ((NSc + C - 1) / C + 3) & ~3), a.slice);
+    const int j0 = min(r * slice, NSc), js1 = min(j0 + slice, NSc);    // my scored blocks [j0, js1)
+    const int jc1 = max(j0, min(js1, NC));                              // my ranked candidates [j0, jc1)
+    for (int j = j0 + tid; j < js1; j += kThreads) {
+        const int pg = page_quiet(c, s, j);
+        pages[j - j0] = pg;
+        if (pg < 0) report(c.status, SBA_DEV_BAD_PAGE);
+    }
     const int k = n_sel - L;
     const bool trivial = k <= 0 || k >= NC;  // take none / all of the candidates
     for (int i = tid; i < L && i < kMaxLocal; i += kThreads) local_page[i] = page_quiet(c, s, NC + i);
@@ -286,41 +292,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (touched_scored) cluster_sync();
 
     // ---------------- phase 1: score this CTA's slice ----------------
-    uint32_t fill = 0;
-    if (warp == kProducer) {
-        for (int j = j0 + lane; j < min(j1, N); j += 32)
-            if (pages[j - j0] < 0) report(c.status, SBA_DEV_BAD_PAGE);
-        const uint8_t* dbase = kScorer == SBA_SCORER_QUEST ? reinterpret_cast<const uint8_t*>(c.desc)
-                                                            : reinterpret_cast<const uint8_t*>(c.kg);
-        bool alive = true;
-        for (int cb = j0; cb < js1; cb += kChunk, ++fill) {
-            const int st = fill % NSt;
-            const int nblk = min(kChunk, js1 - cb);
-            if (lane == 0 && fill >= (uint32_t)NSt && alive)
-                alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
-            alive = __shfl_sync(0xffffffffu, alive, 0);
-            int nv = 0;
-            for (int i = lane; i < nblk; i += 32) nv += pages[cb + i - j0] >= 0;
-            nv = __reduce_add_sync(0xffffffffu, nv);
-            if (lane == 0 && alive) {
-                if (nv > 0)
-                    mbar_arrive_expect_tx(&full[st], nv * kDescBytes);
-                else
-                    mbar_arrive(&full[st]);
-            }
-            __syncwarp();
-            if (alive && nv > 0) {
-                uint8_t* stage = dyn + (size_t)st * TG::kStage;
-                for (int i = lane; i < nblk; i += 32) {
-                    const int pg = pages[cb + i - j0];
-                    if (pg >= 0)
-                        bulk_load(stage + i * kDescBytes, dbase + ((int64_t)pg * c.H_kv + h) * kDescBytes, kDescBytes,
-                                  &full[st]);
-                }
-            }
-        }
-    } else {
-        // consumers: coefficients of this lane's 16-byte chunk of a 512-byte descriptor
+    // Every warp streams descriptors straight into registers: kRB blocks per warp and
+    // round, lane l holding bytes [16 l, 16 l + 16) of each 512-byte descriptor; the
+    // next round's loads are in flight while the current round is reduced.
+    __syncthreads();  // page ids of the slice
+    {
+        constexpr int kNW = kThreads / 32;
+        constexpr int kRB = (kScorer == SBA_SCORER_GATE && kGM > 8) ? 4 : 8;  // (register budget)
+        const uint8_t* src = (kScorer == SBA_SCORER_QUEST ? reinterpret_cast<const uint8_t*>(c.desc)
+                                                          : reinterpret_cast<const uint8_t*>(c.kg)) +
+                             (int64_t)h * kDescBytes + lane * 16;
+        const int64_t pstride = (int64_t)c.H_kv * kDescBytes;
         float coef[8];
         float qg[kGM][4];  // gate: kGM = G rounded up to a power of two
         if (kScorer == SBA_SCORER_QUEST) {
@@ -357,71 +339,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        bool alive = true;
-        const int grp = warp / kGW, gw = warp % kGW;  // consumer group, warp within the group
-        for (int cb = j0; cb < js1; cb += kChunk, ++fill) {
-            if ((int)(fill & 1) != grp) continue;  // the other group's stage
-            const int st = fill % NSt;
-            if (alive) alive = mbar_wait(&full[st], (fill / NSt) & 1, c.status);
-            const int nblk = min(kChunk, js1 - cb);
-            const uint8_t* stage = dyn + (size_t)st * TG::kStage;
+        uint4 wc[kRB], wn[kRB];
+        auto load_round = [&](int base, uint4(&w)[kRB]) {
+#pragma unroll
+            for (int b = 0; b < kRB; ++b) {
+                const int j = base + b;
+                const int pg = j < js1 ? pages[j - j0] : -1;
+                w[b] = pg >= 0 ? ld_stream_v4(src + pg * pstride) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        int base = j0 + warp * kRB;
+        if (base < js1) load_round(base, wc);
+        for (; base < js1; base += kNW * kRB) {
+            if (base + kNW * kRB < js1) load_round(base + kNW * kRB, wn);
             if (kScorer == SBA_SCORER_QUEST) {
-                for (int g8 = gw * 8; g8 < nblk; g8 += kGW * 8) {
-                    float part[8][1];
+                float part[kRB][1];
 #pragma unroll
-                    for (int b8 = 0; b8 < 8; ++b8) {
-                        part[b8][0] = 0.f;
-                        if (g8 + b8 < nblk && alive) {
-                            const uint4 w = *reinterpret_cast<const uint4*>(stage + (g8 + b8) * kDescBytes + lane * 16);
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                            float acc = 0.f;
+                for (int b = 0; b < kRB; ++b) {
+                    const uint32_t ws[4] = {wc[b].x, wc[b].y, wc[b].z, wc[b].w};
+                    float acc = 0.f;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                acc = fmaf(coef[2 * e], bf16_lo(ws[e]), acc);
-                                acc = fmaf(coef[2 * e + 1], bf16_hi(ws[e]), acc);
-                            }
-                            part[b8][0] = acc;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        acc = fmaf(coef[2 * e], bf16_lo(ws[e]), acc);
+                        acc = fmaf(coef[2 * e + 1], bf16_hi(ws[e]), acc);
                     }
-                    float tot[1];
-                    reduce_scatter<8, 1>(part, tot, lane);
-                    const int i = g8 + rs_block<8>(lane);
-                    if ((lane & 3) == 0 && i < nblk) {
-                        const int jl = cb + i - j0;
-                        keys[jl] = pages[jl] >= 0 ? orderable_key(tot[0]) : 0u;
-                    }
+                    part[b][0] = acc;
                 }
+                float tot[1];
+                reduce_scatter<kRB, 1>(part, tot, lane);
+                const int j = base + rs_block<kRB>(lane);
+                if ((lane & 3) == 0 && j < js1) keys[j - j0] = pages[j - j0] >= 0 ? orderable_key(tot[0]) : 0u;
             } else {
-                for (int g4 = gw * 4; g4 < nblk; g4 += kGW * 4) {
+#pragma unroll
+                for (int q4 = 0; q4 < kRB; q4 += 4) {
                     float part[4][kGM];
 #pragma unroll
                     for (int b4 = 0; b4 < 4; ++b4) {
-                        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (g4 + b4 < nblk && alive)
-                            w = *reinterpret_cast<const float4*>(stage + (g4 + b4) * kDescBytes + lane * 16);
+                        const uint4 w = wc[q4 + b4];
+                        const float x0 = __uint_as_float(w.x), x1 = __uint_as_float(w.y), x2 = __uint_as_float(w.z),
+                                    x3 = __uint_as_float(w.w);
 #pragma unroll
                         for (int g = 0; g < kGM; ++g) {
-                            float acc = qg[g][0] * w.x;
-                            acc = fmaf(qg[g][1], w.y, acc);
-                            acc = fmaf(qg[g][2], w.z, acc);
-                            acc = fmaf(qg[g][3], w.w, acc);
+                            float acc = qg[g][0] * x0;
+                            acc = fmaf(qg[g][1], x1, acc);
+                            acc = fmaf(qg[g][2], x2, acc);
+                            acc = fmaf(qg[g][3], x3, acc);
                             part[b4][g] = acc;
                         }
                     }
                     float tot[kGM];
                     reduce_scatter<4, kGM>(part, tot, lane);
-                    const int i = g4 + rs_block<4>(lane);
-                    if ((lane & 7) == 0 && i < nblk) {
-                        const int jl = cb + i - j0;
-                        const bool ok = pages[jl] >= 0;
+                    const int j = base + q4 + rs_block<4>(lane);
+                    if ((lane & 7) == 0 && j < js1) {
+                        const bool ok = pages[j - j0] >= 0;
 #pragma unroll
                         for (int g = 0; g < kGM; ++g)
-                            if (g < G) u_s[g * slice + jl] = ok ? tot[g] : -INFINITY;
+                            if (g < G) u_s[g * ustride + (j - j0)] = ok ? tot[g] : -INFINITY;
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
+#pragma unroll
+            for (int b = 0; b < kRB; ++b) wc[b] = wn[b];
         }
     }
     __syncthreads();
@@ -431,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // per-head (max, sum exp(u - max)) over this CTA's scored blocks, pushed to every CTA
         for (int g = warp; g < G; g += kThreads / 32) {
             float m = -INFINITY;
-            for (int i = lane; i < js1 - j0; i += 32) m = fmaxf(m, u_s[g * slice + i]);
+            for (int i = lane; i < js1 - j0; i += 32) m = fmaxf(m, u_s[g * ustride + i]);
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
@@ -439,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
             float z = 0.f;
             if (m > -INFINITY)
-                for (int i = lane; i < js1 - j0; i += 32) z += expf(u_s[g * slice + i] - m);
+                for (int i = lane; i < js1 - j0; i += 32) z += expf(u_s[g * ustride + i] - m);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
             for (int p = lane; p < C; p += 32) {
@@ -463,20 +441,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // group score of my ranked blocks: sum over the group of g = exp(u - LSE)
         for (int j = j0 + tid; j < jc1; j += kThreads) {
             float sc = 0.f;
-            for (int g = 0; g < G; ++g) sc += expf(u_s[g * slice + (j - j0)] - lse_s[g]);
+            for (int g = 0; g < G; ++g) sc += expf(u_s[g * ustride + (j - j0)] - lse_s[g]);
             keys[j - j0] = pages[j - j0] >= 0 ? orderable_key(sc) : 0u;
         }
         __syncthreads();
     }
     // group size: the largest power of two in [4, 128] leaving >= 2k groups
-    int gs = 128;
+    int gsh = 7;  // log2 of the group size
     if (!trivial)
-        while (gs > 4 && (NC + gs - 1) / gs < 2 * k) gs >>= 1;
-    const int lpg = gs / 4;
-    const int nown = jc1 - j0;                 // my ranked candidates
-    const int ngr = (nown + gs - 1) / gs;      // my groups
-    if (!trivial) {
-        // maxima of my groups (four keys per thread, groups of lpg lanes), pushed to every CTA
+        while (gsh > 2 && ((NC + (1 << gsh) - 1) >> gsh) < 2 * k) --gsh;
+    const int gs = 1 << gsh;
+    // CTA p ranks the blocks [min(p*slice, NC), min(p*slice + slice, NC)) in groups of gs:
+    // every CTA knows every CTA's group count, hence where its maxima go
+    int goff = 0, ng_total = 0;
+    for (int p = 0; p < C; ++p) {
+        const int b0 = min(p * slice, NC);
+        const int ngp = (min(b0 + slice, NC) - b0 + gs - 1) >> gsh;
+        goff += p < r ? ngp : 0;
+        ng_total += ngp;
+    }
+    const int nown = jc1 - j0;  // my ranked candidates
+    if (tid == 0) misc[0] = -1;  // T0 (atomic minimum below)
+    // T0 below is a valid lower bound of the n-th score only when there are >= k groups
+    const bool bound = !trivial && ng_total >= k;
+    // the ranking below reads the maxima as 16-byte vectors: zeros (never larger) pad them
+    const int S_t0 = ng_total * 8 <= kThreads ? 8 : ng_total * 4 <= kThreads ? 4 : ng_total * 2 <= kThreads ? 2 : 1;
+    const int nvec_t0 = (ng_total + 4 * S_t0 - 1) / (4 * S_t0) * S_t0;
+    for (int i = ng_total + tid; i < 4 * nvec_t0; i += kThreads) gmax_all[i] = 0u;
+    if (bound) {
+        // maxima of my groups (four keys per thread, groups of gs/4 lanes), pushed to every CTA
+        const int lpg = gs / 4;
         const uint4* kv = reinterpret_cast<const uint4*>(keys);
         const int nv = (nown + 3) / 4;
         for (int v0 = warp * 32; v0 < nv; v0 += kThreads) {
@@ -490,77 +484,78 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int o = 1; o < lpg; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((lane & (lpg - 1)) == 0 && v < nv) {
-                const int g = v / lpg;
-                for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(gmax_all + r * a.gcap + g, p), m);
+                uint32_t* dst = gmax_all + goff + v / lpg;
+                for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(dst, p), m);
             }
         }
-        for (int p = tid; p < C; p += kThreads) st_peer_u32(peer_addr(&cnt_g[r], p), (uint32_t)ngr);
     }
     cluster_sync();  // every CTA's group maxima pushed
     if (!trivial) {
-        // T0 = smallest group maximum with fewer than k group maxima above it (a valid lower
-        // bound of the n-th score only when there are >= k groups; otherwise take T0 = 0).
-        // The maxima are first packed contiguously (into the crank scratch), then every
-        // thread ranks its maxima against all of them with independent partial counts.
-        uint32_t* gm = reinterpret_cast<uint32_t*>(crank);
-        int ng_total = 0;
-        for (int p = 0; p < C; ++p) ng_total += cnt_g[p];
-        const bool bound = ng_total >= k && ng_total <= a.ccap;
-        if (bound)
-            for (int p = 0, off = 0; p < C; off += cnt_g[p], ++p)
-                for (int g = tid; g < cnt_g[p]; g += kThreads) gm[off + g] = gmax_all[p * a.gcap + g];
-        if (tid == 0) misc[0] = bound ? -1 : 0;
-        __syncthreads();
-        if (bound)
-            for (int g0 = warp * 32; g0 < ng_total; g0 += kThreads) {
-                const int g = g0 + lane;
-                uint32_t cand = 0xffffffffu;
+        uint32_t T0 = 0;
+        if (bound) {
+            // T0 = the k-th largest group maximum (k group maxima are k distinct blocks).  Every
+            // thread counts, for one group maximum, the larger ones among a 1/S share of them.
+            const int S = S_t0;
+            const uint4* gv = reinterpret_cast<const uint4*>(gmax_all);
+            for (int t0 = 0; t0 < ng_total * S; t0 += kThreads) {
+                const int t = t0 + tid, g = t / S, sg = t % S;
+                int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+                uint32_t x = 0;
                 if (g < ng_total) {
-                    const uint32_t x = gm[g];
-                    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-                    int t = 0;
-                    for (; t + 4 <= ng_total; t += 4) {
-                        a0 += gm[t] > x;
-                        a1 += gm[t + 1] > x;
-                        a2 += gm[t + 2] > x;
-                        a3 += gm[t + 3] > x;
+                    x = gmax_all[g];
+#pragma unroll 4
+                    for (int v = sg; v < nvec_t0; v += S) {
+                        const uint4 y = gv[v];
+                        n0 += y.x > x;
+                        n1 += y.y > x;
+                        n2 += y.z > x;
+                        n3 += y.w > x;
                     }
-                    for (; t < ng_total; ++t) a0 += gm[t] > x;
-                    if (a0 + a1 + a2 + a3 < k) cand = x;
                 }
+                int n = (n0 + n1) + (n2 + n3);
+                for (int o = 1; o < S; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+                uint32_t cand = (g < ng_total && n < k) ? x : 0xffffffffu;
                 cand = __reduce_min_sync(0xffffffffu, cand);
                 if (lane == 0 && cand != 0xffffffffu) atomicMin(reinterpret_cast<unsigned*>(&misc[0]), cand);
             }
-        __syncthreads();
-        const uint32_t T0 = (uint32_t)misc[0];
-        // my candidates >= T0 go to my slots [r*cs, r*cs + cs) of every CTA's list,
-        // with their count; a count above cs marks an overflow
-        const int cs = a.ccap / C;
-        if (tid == 0) misc[2] = 0;
-        __syncthreads();
-        for (int i0 = warp * 32; i0 < nown; i0 += kThreads) {
-            const int i = i0 + lane;
-            const bool pass = i < nown && keys[i] >= T0;
-            const unsigned bal = __ballot_sync(0xffffffffu, pass);
-            int off = 0;
-            if (lane == 0 && bal) off = atomicAdd(&misc[2], __popc(bal));
-            off = __shfl_sync(0xffffffffu, off, 0);
-            if (pass) {
-                const int pos = off + __popc(bal & ((1u << lane) - 1u));
-                if (pos < cs) {
-                    const int slot = r * cs + pos;
-                    const uint32_t kk = keys[i];
-                    const int pg = pages[i];
-                    for (int p = 0; p < C; ++p) {
-                        st_peer_u32(peer_addr(ckey + slot, p), kk);
-                        st_peer_u32(peer_addr(cidx + slot, p), (uint32_t)(j0 + i));
-                        st_peer_u32(peer_addr(cpage + slot, p), (uint32_t)pg);
-                    }
-                }
-            }
+            __syncthreads();
+            T0 = (uint32_t)misc[0];
         }
+        // my candidates >= T0, in ascending block order, to my slots [r*cs, r*cs + cs) of every
+        // CTA's list (thread t takes a contiguous run of my keys), then their count (a count
+        // above cs marks an overflow)
+        const int cs = a.ccap / C;
+        const int per = (nown + kThreads - 1) / kThreads;
+        const int i0r = min(tid * per, nown), i1r = min(i0r + per, nown);
+        int cnt = 0;
+        for (int i = i0r; i < i1r; ++i) cnt += keys[i] >= T0;
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
         __syncthreads();
-        for (int p = tid; p < C; p += kThreads) st_peer_u32(peer_addr(&end_all[r], p), (uint32_t)misc[2]);
+        int pos = incl - cnt, total = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            const int x = warp_tot[w];
+            pos += w < warp ? x : 0;
+            total += x;
+        }
+        for (int i = i0r; i < i1r && pos < cs; ++i) {
+            const uint32_t kk = keys[i];
+            if (kk < T0) continue;
+            const int slot = r * cs + pos;
+            const int pg = pages[i];
+            for (int p = 0; p < C; ++p) {
+                st_peer_u32(peer_addr(ckey + slot, p), kk);
+                st_peer_u32(peer_addr(cidx + slot, p), (uint32_t)(j0 + i));
+                st_peer_u32(peer_addr(cpage + slot, p), (uint32_t)pg);
+            }
+            ++pos;
+        }
+        if (tid < C) st_peer_u32(peer_addr(&end_all[r], tid), (uint32_t)total);
     }
     cluster_sync();  // every candidate pushed
     if (trivial) {
@@ -570,55 +565,96 @@ __global__ void __launch_bounds__(kThreads, 1)
             sel_page[i] = first + i >= NC ? local_page[first + i - NC] : -1;
         }
     } else {
-        // the per-source slots, compacted into [0, m) of the idle ring, unless a source overflowed
         const int cs = a.ccap / C;
-        bool overflow = false;
-        int m = 0;
-        for (int p = 0; p < C; ++p) {
-            overflow |= end_all[p] > cs;
-            m += min(end_all[p], cs);
+        // prefix of the per-source counts, and whether a source overflowed
+        if (warp == 0) {
+            const int v = lane < C ? end_all[lane] : 0;
+            const bool ov = __any_sync(0xffffffffu, v > cs);
+            int incl = min(v, cs);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane < C) pre_s[lane + 1] = incl;
+            if (lane == 0) {
+                pre_s[0] = 0;
+                misc[1] = ov;
+            }
         }
+        __syncthreads();
+        const bool overflow = misc[1] != 0;
+        const int m = pre_s[C];
         uint32_t* ck = reinterpret_cast<uint32_t*>(dyn);
-        int* ci = reinterpret_cast<int*>(ck + a.ccap);
-        int* cp = ci + a.ccap;
+        int* ci = reinterpret_cast<int*>(ck + a.ccap + 32);
+        int* cp = ci + a.ccap + 32;
+        const int S = m * 8 <= kThreads ? 8 : m * 4 <= kThreads ? 4 : m * 2 <= kThreads ? 2 : 1;
+        const int nvec = (m + 4 * S - 1) / (4 * S) * S;  // 16-byte vectors of the ranking, padded
         if (!overflow) {
-            for (int p = 0, dst = 0; p < C; dst += end_all[p], ++p)
-                for (int i = tid; i < end_all[p]; i += kThreads) {
-                    ck[dst + i] = ckey[p * cs + i];
-                    ci[dst + i] = cidx[p * cs + i];
-                    cp[dst + i] = cpage[p * cs + i];
-                }
-            __syncthreads();
-        }
-        if (!overflow) {
-            // exact ranks in (key desc, index asc) over the m candidates
+            // the per-source slots, compacted into [0, m) of the idle ring (ascending block order)
             for (int i = tid; i < m; i += kThreads) {
-                const uint32_t ki = ck[i];
-                const int xi = ci[i];
-                int r0 = 0, r1 = 0;
-                int t = 0;
-                for (; t + 2 <= m; t += 2) {
-                    const uint32_t k0 = ck[t], k1 = ck[t + 1];
-                    r0 += (k0 > ki) | ((k0 == ki) & (ci[t] < xi));
-                    r1 += (k1 > ki) | ((k1 == ki) & (ci[t + 1] < xi));
+                int lo = 0, hi = C;  // the source p with pre_s[p] <= i < pre_s[p + 1]
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (pre_s[mid] <= i)
+                        lo = mid;
+                    else
+                        hi = mid;
                 }
-                if (t < m) r0 += (ck[t] > ki) | ((ck[t] == ki) & (ci[t] < xi));
-                crank[i] = r0 + r1;
+                const int slot = lo * cs + (i - pre_s[lo]);
+                ck[i] = ckey[slot];
+                ci[i] = cidx[slot];
+                cp[i] = cpage[slot];
+            }
+            for (int i = m + tid; i < 4 * nvec; i += kThreads) {  // pads rank below everything
+                ck[i] = 0u;
+                ci[i] = 0x7fffffff;
             }
             __syncthreads();
-            for (int i = tid; i < m; i += kThreads) {
-                if (crank[i] >= k) continue;
-                const int xi = ci[i];
-                int p0c = 0, p1c = 0;
-                int t = 0;
-                for (; t + 2 <= m; t += 2) {
-                    p0c += (crank[t] < k) & (ci[t] < xi);
-                    p1c += (crank[t + 1] < k) & (ci[t + 1] < xi);
+            // exact rank in (key desc, index asc) of every candidate, S threads per candidate
+            const uint4* kv4 = reinterpret_cast<const uint4*>(ck);
+            const int4* iv4 = reinterpret_cast<const int4*>(ci);
+            for (int t0 = 0; t0 < m * S; t0 += kThreads) {
+                const int t = t0 + tid, i = t / S, sg = t % S;
+                int n0 = 0, n1 = 0;
+                if (i < m) {
+                    const uint32_t ki = ck[i];
+                    const int xi = ci[i];
+#pragma unroll 2
+                    for (int v = sg; v < nvec; v += S) {
+                        const uint4 y = kv4[v];
+                        const int4 z = iv4[v];
+                        n0 += (y.x > ki) | ((y.x == ki) & (z.x < xi));
+                        n1 += (y.y > ki) | ((y.y == ki) & (z.y < xi));
+                        n0 += (y.z > ki) | ((y.z == ki) & (z.z < xi));
+                        n1 += (y.w > ki) | ((y.w == ki) & (z.w < xi));
+                    }
                 }
-                if (t < m) p0c += (crank[t] < k) & (ci[t] < xi);
-                const int pos = p0c + p1c;
-                sel[pos] = xi;
-                sel_page[pos] = cp[i];
+                int n = n0 + n1;
+                for (int o = 1; o < S; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+                if (i < m && sg == 0) crank[i] = n;
+            }
+            __syncthreads();
+            // the k best, in ascending block order: output position = selected ones before
+            for (int t0 = 0, run = 0; t0 < m; t0 += kThreads) {
+                const int i = t0 + tid;
+                const bool take = i < m && crank[i] < k;
+                const unsigned bal = __ballot_sync(0xffffffffu, take);
+                if (lane == 0) warp_tot[warp] = __popc(bal);
+                __syncthreads();
+                int off = run, tot = 0;
+                for (int w = 0; w < kThreads / 32; ++w) {
+                    const int x = warp_tot[w];
+                    off += w < warp ? x : 0;
+                    tot += x;
+                }
+                if (take) {
+                    const int p = off + __popc(bal & ((1u << lane) - 1u));
+                    sel[p] = ci[i];
+                    sel_page[p] = cp[i];
+                }
+                run += tot;
+                __syncthreads();
             }
         } else {
             // too many candidates (e.g. many equal scores): gather every score into the idle
@@ -656,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------- phase 3: decode this CTA's share of the selection ----------------
+    uint32_t fill = 0;  // ring fills so far (consecutive fills alternate consumer groups)
     const int i0 = (int)((int64_t)n_sel * r / C), i1 = (int)((int64_t)n_sel * (r + 1) / C);
     const bool tile_refresh = n_new > 0 && !touched_scored;
     const int E = G * kHeadDim;         // merge elements (row, channel) of this group
@@ -720,8 +757,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float b0 = 0.f, b1 = 0.f;
                 if (kScorer == SBA_SCORER_GATE && inf.j != N - 1) {
                     const int owner = inf.j / slice, off = inf.j - owner * slice;
-                    if (rr < G) b0 = ld_peer_f32(peer_addr(u_s + rr * slice + off, owner)) - lse_s[rr];
-                    if (rr + 8 < G) b1 = ld_peer_f32(peer_addr(u_s + (rr + 8) * slice + off, owner)) - lse_s[rr + 8];
+                    if (rr < G) b0 = ld_peer_f32(peer_addr(u_s + rr * ustride + off, owner)) - lse_s[rr];
+                    if (rr + 8 < G) b1 = ld_peer_f32(peer_addr(u_s + (rr + 8) * ustride + off, owner)) - lse_s[rr + 8];
                 }
                 if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && (lane & 3) == 0 && inf.pos < a.n_max) {
                     if (rr < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr) * a.n_max + inf.pos] = b0;
@@ -778,16 +815,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&empty[st]);
         }
         named_sync(3, kCW * 32);  // every consumer is done with the ring before it becomes the merge area
-        decode_state_store(dst, merge_o, merge_ml, warp, lane);
+        decode_state_store(dst, merge_o, merge_ml, warp, lane, G);
         named_sync(3, kCW * 32);
-        // this CTA's partial (O, LSE) of every element, pushed to the element's merging CTA
+        // per query row: the weight of each consumer warp's partial and the row's LSE over this
+        // CTA's blocks (pushed to every CTA); kCW consecutive lanes per row
+        if (warp < (G * kCW + 31) / 32) {  // whole warps: every lane takes part in the shuffles
+            const int row = tid / kCW, w = tid % kCW;
+            const bool act = row < G;  // (rows come in groups of kCW lanes)
+            const float mw = act ? merge_ml[(w * 16 + row) * 2] : -INFINITY;
+            const float lw = act ? merge_ml[(w * 16 + row) * 2 + 1] : 0.f;
+            float M = mw;
+#pragma unroll
+            for (int o = 1; o < kCW; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            float ls = f * lw;
+#pragma unroll
+            for (int o = 1; o < kCW; o <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+            if (act) {
+                wgt_s[row][w] = ls > 0.f ? f / ls : 0.f;
+                const float lse = ls > 0.f ? (M + log2f(ls)) * kLn2 : -INFINITY;
+                for (int p = w; p < C; p += kCW) st_peer_f32(peer_addr(&lse_all[r * G + row], p), lse);
+            }
+        }
+        named_sync(3, kCW * 32);
+        // this CTA's normalised partial O of every element, pushed to the element's merging CTA
         for (int e = tid; e < E; e += kCW * 32) {
             const int row = e / kHeadDim, ch = e % kHeadDim;
-            float o, lse;
-            merge_warps(merge_o, merge_ml, row, ch, o, lse, kCW);
+            const float4 w0 = *reinterpret_cast<const float4*>(&wgt_s[row][0]);
+            const float4 w1 = *reinterpret_cast<const float4*>(&wgt_s[row][4]);
+            const float* mo = merge_o + row * kHeadDim + ch;
+            float o = w0.x * mo[0];
+            o = fmaf(w0.y, mo[1 * 16 * kHeadDim], o);
+            o = fmaf(w0.z, mo[2 * 16 * kHeadDim], o);
+            o = fmaf(w0.w, mo[3 * 16 * kHeadDim], o);
+            o = fmaf(w1.x, mo[4 * 16 * kHeadDim], o);
+            o = fmaf(w1.y, mo[5 * 16 * kHeadDim], o);
+            o = fmaf(w1.z, mo[6 * 16 * kHeadDim], o);
+            o = fmaf(w1.w, mo[7 * 16 * kHeadDim], o);
             const int p = e / share;
             st_peer_f32(peer_addr(recv_o + r * share + (e - p * share), p), o);
-            if (ch < C) st_peer_f32(peer_addr(&lse_all[r * G + row], ch), lse);
         }
     }
 
@@ -871,7 +937,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + (c.b == 64 ? 1 : 0);
     int ns = 6;
     const int fixed_bytes = 4 * (round4(pl.slice) * 2 + (p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0) +
-                                 C * pl.gcap + 4 * pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
+                                 C * pl.gcap + 32 + 4 * pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
     const int budget = 227 * 1024 - 1024 /*align*/ - 8 * 1024 /*static shared memory headroom*/;
     while (ns > max(2, min_stages) && ns * stage + fixed_bytes + ns * (16 + (int)sizeof(StageInfo)) > budget) --ns;
     pl.n_stages = ns;
@@ -879,7 +945,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     pl.off_keys = take(pl.slice);
     pl.off_pages = take(pl.slice);
     pl.off_u = take(p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0);
-    pl.off_gmax = take(C * pl.gcap);
+    pl.off_gmax = take(C * pl.gcap + 32);
     pl.off_ckey = take(pl.ccap);
     pl.off_cidx = take(pl.ccap);
     pl.off_cpage = take(pl.ccap);
