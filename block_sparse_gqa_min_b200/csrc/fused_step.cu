@@ -172,6 +172,85 @@ __device__ void refresh_from_global(const StepArgs& a, int s, int h, int j, int 
     }
 }
 
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Descriptor of a touched block from its K tile staged in shared memory, by one warp:
+// lane = 16-byte chunk (8 channels) of a row x token parity.  Quest: the min/max rows
+// (exact in bf16) go to the cache; gate: the pooled [max | min | avg] summary is pushed
+// to every CTA of the cluster, which project it after the merge.
+template <int kBlk, int kScorer>
+__device__ __forceinline__ void refresh_from_stage(const sba_cache& c, const uint8_t* stage, int valid, int64_t pg,
+                                                   int h, float* pooled_b0, int C, int lane) {
+    using TG = TileGeom<kBlk>;
+    const int ck = lane & 15, cc = ck & 7;
+    const uint8_t* kt = stage + (ck >> 3) * TG::kHalf;
+    uint32_t mn[4], mx[4];
+    float sm[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        mn[e] = 0x7f807f80u;  // +inf, +inf
+        mx[e] = 0xff80ff80u;  // -inf, -inf
+        sm[2 * e] = sm[2 * e + 1] = 0.f;
+    }
+#pragma unroll 4
+    for (int t = lane >> 4; t < valid; t += 2) {
+        const uint4 w = *reinterpret_cast<const uint4*>(kt + t * 128 + ((cc ^ (t & 7)) << 4));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            mn[e] = bf16x2_min(mn[e], ws[e]);
+            mx[e] = bf16x2_max(mx[e], ws[e]);
+            if (kScorer == SBA_SCORER_GATE) {
+                sm[2 * e] += bf16_lo(ws[e]);
+                sm[2 * e + 1] += bf16_hi(ws[e]);
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {  // the other token parity
+        mn[e] = bf16x2_min(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], 16));
+        mx[e] = bf16x2_max(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
+        if (kScorer == SBA_SCORER_GATE) {
+            sm[2 * e] += __shfl_xor_sync(0xffffffffu, sm[2 * e], 16);
+            sm[2 * e + 1] += __shfl_xor_sync(0xffffffffu, sm[2 * e + 1], 16);
+        }
+    }
+    if (lane >= 16) return;
+    if (kScorer == SBA_SCORER_QUEST) {
+        uint8_t* d = reinterpret_cast<uint8_t*>(c.desc) + (pg * c.H_kv + h) * 2 * kHeadDim * 2;
+        *reinterpret_cast<uint4*>(d + ck * 16) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
+        *reinterpret_cast<uint4*>(d + 2 * kHeadDim + ck * 16) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
+    } else {
+        const float inv = 1.f / (float)valid;
+        const float4 hi0 = make_float4(bf16_lo(mx[0]), bf16_hi(mx[0]), bf16_lo(mx[1]), bf16_hi(mx[1]));
+        const float4 hi1 = make_float4(bf16_lo(mx[2]), bf16_hi(mx[2]), bf16_lo(mx[3]), bf16_hi(mx[3]));
+        const float4 lo0 = make_float4(bf16_lo(mn[0]), bf16_hi(mn[0]), bf16_lo(mn[1]), bf16_hi(mn[1]));
+        const float4 lo1 = make_float4(bf16_lo(mn[2]), bf16_hi(mn[2]), bf16_lo(mn[3]), bf16_hi(mn[3]));
+        const float4 av0 = make_float4(sm[0] * inv, sm[1] * inv, sm[2] * inv, sm[3] * inv);
+        const float4 av1 = make_float4(sm[4] * inv, sm[5] * inv, sm[6] * inv, sm[7] * inv);
+        auto bits = [](float4 v) {
+            return make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w));
+        };
+        for (int p = 0; p < C; ++p) {
+            st_peer_v4(peer_addr(pooled_b0 + 8 * ck, p), bits(hi0));
+            st_peer_v4(peer_addr(pooled_b0 + 8 * ck + 4, p), bits(hi1));
+            st_peer_v4(peer_addr(pooled_b0 + kHeadDim + 8 * ck, p), bits(lo0));
+            st_peer_v4(peer_addr(pooled_b0 + kHeadDim + 8 * ck + 4, p), bits(lo1));
+            st_peer_v4(peer_addr(pooled_b0 + 2 * kHeadDim + 8 * ck, p), bits(av0));
+            st_peer_v4(peer_addr(pooled_b0 + 2 * kHeadDim + 8 * ck + 4, p), bits(av1));
+        }
+    }
+}
+
 // Physical page of block j without reporting (speculative lookups).
 __device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
     const int64_t p = c.block_table ? (int64_t)__ldg(c.block_table + (int64_t)s * c.max_blocks + j)
@@ -709,11 +788,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         bool alive = true;
+        // blocks touched by this step's append get their descriptors from the staged K tiles
+        // here, before their stage is reused or, for the last NSt positions, after the loop
+        auto touched = [&](int i) {
+            const int j = sel[i];
+            return tile_refresh && j >= tb0 && j <= tb1 && sel_page[i] >= 0;
+        };
+        auto refresh = [&](int i, int st) {
+            const int j = sel[i];
+            refresh_from_stage<kBlk, kScorer>(c, dyn + (size_t)st * TG::kStage, min(kBlk, len - j * kBlk),
+                                              sel_page[i], h, pooled_b0, C, lane);
+            fence_proxy_async_smem();  // these generic reads before the next TMA write of the stage
+            __syncwarp();
+        };
         for (int i = i0; i < i1; ++i, ++fill) {
             const int st = fill % NSt;
+            if (fill >= (uint32_t)NSt) {
+                if (lane == 0 && alive) alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
+                alive = __shfl_sync(0xffffffffu, alive, 0);
+                if (alive && touched(i - NSt)) {
+                    bool ok = true;  // (complete: the consumers released it)
+                    if (lane == 0) ok = mbar_wait(&full[st], ((fill / NSt) - 1) & 1, c.status);
+                    if (__shfl_sync(0xffffffffu, ok, 0)) refresh(i - NSt, st);
+                }
+            }
             if (lane == 0 && alive) {
-                if (fill >= (uint32_t)NSt) alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
-                if (alive) {
+                {
                     const int j = sel[i];
                     const int pg = (j >= 0 && j < N) ? sel_page[i] : -1;
                     StageInfo inf;
@@ -738,6 +838,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
         }
+        for (int i = max(i0, i1 - NSt); i < i1; ++i) {
+            if (!alive || !touched(i)) continue;
+            const uint32_t f = (uint32_t)(i - i0);
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&full[f % NSt], (f / NSt) & 1, c.status);
+            if (__shfl_sync(0xffffffffu, ok, 0)) refresh(i, (int)(f % NSt));
+        }
+        named_sync(4, kThreads);  // the ring becomes the merge area
     } else {
         uint32_t qa[8][4];
         load_q_frags(qa, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
@@ -766,55 +874,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (alive)
                     decode_block<kBlk>(dst, qa, stage, inf.valid, b0 * kLog2e, b1 * kLog2e, a.scale_log2, gw, lane);
-                // (the condition below depends only on the stage info, the same for all four warps)
-                if (tile_refresh && inf.j >= tb0 && inf.j <= tb1) {
-                    // descriptor of a touched (local) block from its staged K tile (the group's
-                    // 128 threads, one channel each)
-                    named_sync(1 + grp, kGW * 32);
-                    const int ch = tid - grp * kGW * 32;
-                    const uint8_t* khalf = stage + (ch >> 6) * TG::kHalf;
-                    const int cc = (ch & 63) >> 3, e = ch & 7;
-                    float lo4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
-                    float hi4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    float sm4[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int t0 = 0; t0 < inf.valid; t0 += 4) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int t = t0 + u;
-                            if (t < inf.valid) {
-                                const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                    khalf + t * 128 + ((cc ^ (t & 7)) << 4) + e * 2));
-                                lo4[u] = fminf(lo4[u], x);
-                                hi4[u] = fmaxf(hi4[u], x);
-                                sm4[u] += x;
-                            }
-                        }
-                    }
-                    const float lo = fminf(fminf(lo4[0], lo4[1]), fminf(lo4[2], lo4[3]));
-                    const float hi = fmaxf(fmaxf(hi4[0], hi4[1]), fmaxf(hi4[2], hi4[3]));
-                    const float sum = (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
-                    const int64_t pg = sel_page[inf.pos];
-                    if (kScorer == SBA_SCORER_QUEST) {
-                        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(c.desc) + (pg * c.H_kv + h) * 2 * kHeadDim;
-                        d[ch] = __float2bfloat16_rn(lo);
-                        d[kHeadDim + ch] = __float2bfloat16_rn(hi);
-                    } else {
-                        // pooled summary of the current block, pushed to every CTA for the projection
-                        const float avg = sum / (float)inf.valid;
-                        for (int p = 0; p < C; ++p) {
-                            st_peer_f32(peer_addr(&pooled_b0[ch], p), hi);
-                            st_peer_f32(peer_addr(&pooled_b0[kHeadDim + ch], p), lo);
-                            st_peer_f32(peer_addr(&pooled_b0[2 * kHeadDim + ch], p), avg);
-                        }
-                    }
-                    named_sync(1 + grp, kGW * 32);
-                }
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
-        named_sync(3, kCW * 32);  // every consumer is done with the ring before it becomes the merge area
+        named_sync(4, kThreads);  // every consumer (and the producer) is done with the ring: it becomes the merge area
         decode_state_store(dst, merge_o, merge_ml, warp, lane, G);
         named_sync(3, kCW * 32);
         // per query row: the weight of each consumer warp's partial and the row's LSE over this
