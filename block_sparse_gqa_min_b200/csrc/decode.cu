@@ -256,6 +256,22 @@ bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Descriptor rows (512 bytes per (page, KV head)) of a contiguous cache as a 4-D
+// map of 4-byte words: 32 words x 4 quarter rows x H_kv x pages, one box = `rows`
+// consecutive pages of one head, 128-byte swizzle (16-byte chunk c of quarter row R
+// lands at chunk c ^ (R & 7)).
+bool make_desc_tmap(CUtensorMap* m, void* base, uint64_t pages, int H_kv, int rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {32, 4, (cuuint64_t)H_kv, pages};
+    cuuint64_t strides[3] = {128, 512, (cuuint64_t)H_kv * 512};
+    cuuint32_t box[4] = {32, 4, 1, (cuuint32_t)rows};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 template <int kBlk>

@@ -37,7 +37,8 @@
 
 namespace sba {
 
-bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);  // decode.cu
+bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);                // decode.cu
+bool make_desc_tmap(CUtensorMap* m, void* base, uint64_t pages, int H_kv, int rows);  // decode.cu
 
 namespace {
 
@@ -119,18 +120,23 @@ __device__ __forceinline__ int rs_block(int lane) {
 }
 
 // CTA 0: write the step's new tokens of (s, h) into the cache.
-__device__ void append_rows(const StepArgs& a, int s, int h, int p0, int tid) {
+// Element e of the step's new rows of (s, h): per token 16 x 16 B of K, then 16 x 16 B of V.
+__device__ __forceinline__ const uint4* append_src(const StepArgs& a, int s, int h, int e) {
+    const int tok = e >> 5, half = (e >> 4) & 1, l = e & 15;
+    return (half ? a.v_new : a.k_new) + (((int64_t)s * a.n_new + tok) * a.c.H_kv + h) * 16 + l;
+}
+__device__ __forceinline__ void append_store(const StepArgs& a, int s, int h, int p0, int e, uint4 v) {
     const sba_cache& c = a.c;
-    const int total = a.n_new * 32;  // per token: 16 x 16 B of K, 16 x 16 B of V
-    for (int e = tid; e < total; e += kThreads) {
-        const int tok = e >> 5, half = (e >> 4) & 1, l = e & 15;
-        const int pos = p0 + tok;
-        const int64_t page = page_of(c, s, pos / c.b, c.status);
-        if (page < 0) continue;
-        const uint4* src = (half ? a.v_new : a.k_new) + (((int64_t)s * a.n_new + tok) * c.H_kv + h) * 16 + l;
-        uint4* dst = reinterpret_cast<uint4*>(half ? c.v : c.k) + ((page * c.H_kv + h) * c.b + pos % c.b) * 16 + l;
-        *dst = __ldg(src);
-    }
+    const int tok = e >> 5, half = (e >> 4) & 1, l = e & 15;
+    const int pos = p0 + tok;
+    const int64_t page = page_of(c, s, pos / c.b, c.status);
+    if (page < 0) return;
+    reinterpret_cast<uint4*>(half ? c.v : c.k)[((page * c.H_kv + h) * c.b + pos % c.b) * 16 + l] = v;
+}
+
+// Elements [e0, e1) of the step's new rows, written through the block table.
+__device__ void append_rows(const StepArgs& a, int s, int h, int p0, int e0, int e1, int tid) {
+    for (int e = e0 + tid; e < e1; e += kThreads) append_store(a, s, h, p0, e, __ldg(append_src(a, s, h, e)));
     fence_proxy_async_global();
 }
 
@@ -251,6 +257,26 @@ __device__ __forceinline__ void refresh_from_stage(const sba_cache& c, const uin
     }
 }
 
+// Quest weights of this lane's 16 bytes of a descriptor: lane < 16 holds MIN row channels
+// 8*lane..+7 (weight M = sum over the group's heads of min(q, 0)); lane >= 16 the MAX row
+// channels 8*(lane-16)..+7 (weight P = sum of max(q, 0)).
+__device__ __forceinline__ void quest_coef(float (&coef)[8], const __nv_bfloat16* qg, int G, int lane) {
+    const int ch0 = (lane & 15) * 8;
+    const bool use_max = lane >= 16;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) coef[e] = 0.f;
+    for (int g = 0; g < G; ++g) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)g * kHeadDim + ch0));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = bf16_lo(ws[e]), x1 = bf16_hi(ws[e]);
+            coef[2 * e] += use_max ? fmaxf(x0, 0.f) : fminf(x0, 0.f);
+            coef[2 * e + 1] += use_max ? fmaxf(x1, 0.f) : fminf(x1, 0.f);
+        }
+    }
+}
+
 // Physical page of block j without reporting (speculative lookups).
 __device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
     const int64_t p = c.block_table ? (int64_t)__ldg(c.block_table + (int64_t)s * c.max_blocks + j)
@@ -260,7 +286,8 @@ __device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
 
 template <int kBlk, int kScorer, int kGM>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, StepArgs a) {
+    decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmD, StepArgs a) {
     using TG = TileGeom<kBlk>;
     constexpr int kMaxLocal = 64;
     __shared__ uint32_t hist[256];
@@ -316,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kProducer && lane == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
+        if (c.block_table == nullptr) prefetch_tmap(&tmD);
     }
     __syncthreads();
     pdl_wait();
@@ -360,22 +388,197 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool touched_scored = n_new > 0 && tb0 <= tb1 && tb0 < NSc;
 
     // ---------------- append (and, if needed, refresh before scoring) ----------------
-    if (r == 0 && n_new > 0) {
-        append_rows(a, s, h, p0, tid);
-        if (touched_scored) {
+    // When a touched block is scored, CTA 0 writes the new rows and refreshes those blocks
+    // before anyone scores.  Otherwise each CTA loads its share of the rows now (one element
+    // per thread; a share above the CTA's threads is written at once) and stores it after
+    // scoring, before the cluster barriers that order it ahead of the decode's tile loads.
+    uint4 app_v = make_uint4(0u, 0u, 0u, 0u);
+    int app_e = -1;
+    if (touched_scored) {
+        if (r == 0) {
+            append_rows(a, s, h, p0, 0, n_new * 32, tid);
             __syncthreads();
             for (int j = tb0; j <= tb1; ++j) refresh_from_global<kScorer>(a, s, h, j, len, pooled, tid);
             fence_proxy_async_global();
         }
+        cluster_sync();
+    } else if (n_new > 0) {
+        const int total = n_new * 32, per = (total + C - 1) / C;
+        const int e0 = min(r * per, total), e1 = min(e0 + per, total);
+        if (e0 + tid < e1) {
+            app_e = e0 + tid;
+            app_v = __ldg(append_src(a, s, h, app_e));
+        }
+        if (e1 - e0 > kThreads) append_rows(a, s, h, p0, e0 + kThreads, e1, tid);
     }
-    if (touched_scored) cluster_sync();
 
     // ---------------- phase 1: score this CTA's slice ----------------
-    // Every warp streams descriptors straight into registers: kRB blocks per warp and
-    // round, lane l holding bytes [16 l, 16 l + 16) of each 512-byte descriptor; the
-    // next round's loads are in flight while the current round is reduced.
     __syncthreads();  // page ids of the slice
-    {
+    uint32_t fill = 0;  // ring fills so far (consecutive fills alternate consumer groups)
+    if (c.block_table == nullptr) {
+        // Contiguous cache: one TMA load brings the descriptors of kBlk consecutive blocks into
+        // a ring stage (128-byte quarter rows, 128-byte swizzle); the two consumer groups take
+        // alternate stages, each warp 16 descriptors (one tensor-core tile for the gate) per
+        // 64 of the stage.
+        const int nch = (js1 - j0 + kBlk - 1) / kBlk;
+        if (warp == kProducer) {
+            if (lane == 0) {
+                bool alive = true;
+                for (int f = 0; f < nch && alive; ++f) {
+                    const int st = f % NSt;
+                    if (f >= NSt) alive = mbar_wait(&empty[st], ((f / NSt) - 1) & 1, c.status);
+                    if (alive) {
+                        mbar_arrive_expect_tx(&full[st], TG::kStage);
+                        tma_load_4d(dyn + (size_t)st * TG::kStage, &tmD, &full[st], 0, 0, h, s * mb + j0 + f * kBlk);
+                    }
+                }
+            }
+        } else {
+            const int grp = warp / kGW, gw = warp % kGW;
+            constexpr int kIt = kBlk / 64;         // 16-descriptor pieces of a stage per warp
+            constexpr int NTq = kGM > 8 ? 2 : 1;  // gate: 8-head n-tiles
+            float coef[8];
+            uint32_t qf[NTq][8][4];
+            if (kScorer == SBA_SCORER_QUEST) {
+                quest_coef(coef, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
+            } else {
+                // B fragments: head nt*8 + lane/4, channels 16p + 4(lane%4) + 0..3 (bf16 is exact in tf32)
+#pragma unroll
+                for (int nt = 0; nt < NTq; ++nt) {
+                    const int head = nt * 8 + (lane >> 2);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        uint2 w = make_uint2(0u, 0u);
+                        if (head < G)
+                            w = __ldg(reinterpret_cast<const uint2*>(a.q + ((int64_t)s * c.H_q + h * G + head) * kHeadDim +
+                                                                    16 * p + 4 * (lane & 3)));
+                        qf[nt][p][0] = w.x << 16;
+                        qf[nt][p][1] = w.x & 0xffff0000u;
+                        qf[nt][p][2] = w.y << 16;
+                        qf[nt][p][3] = w.y & 0xffff0000u;
+                    }
+                }
+            }
+            bool alive = true;
+            for (int f = grp; f < nch; f += kGroups) {
+                const int st = f % NSt;
+                if (alive) alive = mbar_wait(&full[st], (f / NSt) & 1, c.status);
+                const int cb = j0 + f * kBlk, nblk = min(kBlk, js1 - cb);
+                const uint8_t* stage = dyn + (size_t)st * TG::kStage;
+                if (kScorer == SBA_SCORER_QUEST) {
+#pragma unroll
+                    for (int it = 0; it < kIt; ++it) {
+                        // two independent rounds of 8 descriptors, lane l = bytes [16 l, 16 l + 16) of each
+                        const int n0 = 16 * gw + 64 * it;
+                        if (n0 >= nblk) break;
+                        float part[2][8][1];
+#pragma unroll
+                        for (int rd = 0; rd < 2; ++rd)
+#pragma unroll
+                            for (int b8 = 0; b8 < 8; ++b8) {
+                                const int R = (n0 + 8 * rd + b8) * 4 + (lane >> 3);
+                                const uint4 w =
+                                    *reinterpret_cast<const uint4*>(stage + R * 128 + (((lane & 7) ^ (R & 7)) << 4));
+                                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                                float acc = 0.f;
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    acc = fmaf(coef[2 * e], bf16_lo(ws[e]), acc);
+                                    acc = fmaf(coef[2 * e + 1], bf16_hi(ws[e]), acc);
+                                }
+                                part[rd][b8][0] = acc;
+                            }
+                        float tot[2][1];
+                        reduce_scatter<8, 1>(part[0], tot[0], lane);
+                        reduce_scatter<8, 1>(part[1], tot[1], lane);
+#pragma unroll
+                        for (int rd = 0; rd < 2; ++rd) {
+                            const int i = n0 + 8 * rd + rs_block<8>(lane);
+                            if ((lane & 3) == 0 && i < nblk) {
+                                const int jl = cb + i - j0;
+                                keys[jl] = pages[jl] >= 0 ? orderable_key(tot[rd][0]) : 0u;
+                            }
+                        }
+                    }
+                } else {
+                    // u = q . kg on tensor cores: tiles of 16 blocks (rows) x 8 heads (columns);
+                    // kg = hi + lo in tf32 (hi = kg rounded, lo = the rounded remainder); four
+                    // accumulators per tile (channel half x hi/lo) keep the MMA chains short, and
+                    // a warp's tiles of the stage run interleaved when registers allow
+                    constexpr int kTl = (kIt == 2 && NTq == 1) ? 2 : 1;
+                    const int gq = lane >> 2, t = lane & 3;
+#pragma unroll
+                    for (int it0 = 0; it0 < kIt; it0 += kTl) {
+                        if (16 * gw + 64 * it0 >= nblk) break;
+                        float acc[kTl][NTq][4][4];
+#pragma unroll
+                        for (int tl = 0; tl < kTl; ++tl)
+#pragma unroll
+                            for (int nt = 0; nt < NTq; ++nt)
+#pragma unroll
+                                for (int x = 0; x < 4; ++x)
+                                    acc[tl][nt][x][0] = acc[tl][nt][x][1] = acc[tl][nt][x][2] = acc[tl][nt][x][3] = 0.f;
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+#pragma unroll
+                            for (int tl = 0; tl < kTl; ++tl) {
+                                const int n0 = 16 * gw + 64 * (it0 + tl);
+                                const int R0 = (n0 + gq) * 4 + (p >> 1);
+                                const int off = ((((p & 1) << 2) | t) ^ (R0 & 7)) << 4;
+                                const float4 x0 = *reinterpret_cast<const float4*>(stage + R0 * 128 + off);
+                                const float4 x1 = *reinterpret_cast<const float4*>(stage + (R0 + 32) * 128 + off);
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const float v[4] = {e ? x0.z : x0.x, e ? x1.z : x1.x, e ? x0.w : x0.y,
+                                                        e ? x1.w : x1.y};
+                                    uint32_t hi[4], lo[4];
+#pragma unroll
+                                    for (int u = 0; u < 4; ++u) {
+                                        hi[u] = to_tf32(v[u]);
+                                        lo[u] = to_tf32(v[u] - __uint_as_float(hi[u]));
+                                    }
+                                    const int ah = (p >> 2) * 2;  // accumulator pair of this channel half
+#pragma unroll
+                                    for (int nt = 0; nt < NTq; ++nt) {
+                                        mma_tf32_1688(acc[tl][nt][ah], hi, qf[nt][p][2 * e], qf[nt][p][2 * e + 1]);
+                                        mma_tf32_1688(acc[tl][nt][ah + 1], lo, qf[nt][p][2 * e], qf[nt][p][2 * e + 1]);
+                                    }
+                                }
+                            }
+                        }
+                        // u of blocks n0 + gq (elements 0, 1) and n0 + gq + 8 (2, 3), heads nt*8 + 2t (+1)
+#pragma unroll
+                        for (int tl = 0; tl < kTl; ++tl)
+#pragma unroll
+                            for (int hb = 0; hb < 2; ++hb) {
+                                const int i = 16 * gw + 64 * (it0 + tl) + gq + 8 * hb;
+                                if (i < nblk) {
+                                    const int jl = cb + i - j0;
+                                    const bool ok = pages[jl] >= 0;
+#pragma unroll
+                                    for (int nt = 0; nt < NTq; ++nt)
+#pragma unroll
+                                        for (int x = 0; x < 2; ++x) {
+                                            const int hd = nt * 8 + 2 * t + x, el = 2 * hb + x;
+                                            const float u = (acc[tl][nt][0][el] + acc[tl][nt][2][el]) +
+                                                            (acc[tl][nt][1][el] + acc[tl][nt][3][el]);
+                                            if (hd < G) u_s[hd * ustride + jl] = ok ? u : -INFINITY;
+                                        }
+                                }
+                            }
+                    }
+                }
+                fence_proxy_async_smem();  // these reads before the next TMA write of the stage
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+        }
+        fill = (uint32_t)nch;
+    } else {
+    // Paged cache: every warp streams descriptors straight into registers: kRB blocks per
+    // warp and round, lane l holding bytes [16 l, 16 l + 16) of each 512-byte descriptor;
+    // the next round's loads are in flight while the current round is reduced.
+
         constexpr int kNW = kThreads / 32;
         constexpr int kRB = (kScorer == SBA_SCORER_GATE && kGM > 8) ? 4 : 8;  // (register budget)
         const uint8_t* src = (kScorer == SBA_SCORER_QUEST ? reinterpret_cast<const uint8_t*>(c.desc)
@@ -385,23 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float coef[8];
         float qg[kGM][4];  // gate: kGM = G rounded up to a power of two
         if (kScorer == SBA_SCORER_QUEST) {
-            // chunk lane < 16: MIN row channels 8*lane..+7 (weights M = sum_qh min(q,0));
-            // lane >= 16: MAX row channels 8*(lane-16)..+7 (weights P = sum_qh max(q,0))
-            const int ch0 = (lane & 15) * 8;
-            const bool use_max = lane >= 16;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) coef[e] = 0.f;
-            for (int g = 0; g < G; ++g) {
-                const uint4 w =
-                    __ldg(reinterpret_cast<const uint4*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim + ch0));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = bf16_lo(ws[e]), x1 = bf16_hi(ws[e]);
-                    coef[2 * e] += use_max ? fmaxf(x0, 0.f) : fminf(x0, 0.f);
-                    coef[2 * e + 1] += use_max ? fmaxf(x1, 0.f) : fminf(x1, 0.f);
-                }
-            }
+            quest_coef(coef, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
         } else {
             // gate: lane owns channels 4*lane..4*lane+3 of the fp32 gate key
 #pragma unroll
@@ -482,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     __syncthreads();
+    if (app_e >= 0) append_store(a, s, h, p0, app_e, app_v);  // (its proxy fence comes before barrier B)
 
     // ---------------- phase 2: distributed selection ----------------
     if (kScorer == SBA_SCORER_GATE) {
@@ -636,6 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (tid < C) st_peer_u32(peer_addr(&end_all[r], tid), (uint32_t)total);
     }
+    if (app_e >= 0) fence_proxy_async_global();  // the appended rows, for the decode's tile loads
     cluster_sync();  // every candidate pushed
     if (trivial) {
         const int first = k <= 0 ? NC : 0;
@@ -771,7 +960,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---------------- phase 3: decode this CTA's share of the selection ----------------
-    uint32_t fill = 0;  // ring fills so far (consecutive fills alternate consumer groups)
     const int i0 = (int)((int64_t)n_sel * r / C), i1 = (int)((int64_t)n_sel * (r + 1) / C);
     const bool tile_refresh = n_new > 0 && !touched_scored;
     const int E = G * kHeadDim;         // merge elements (row, channel) of this group
@@ -801,12 +989,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();  // these generic reads before the next TMA write of the stage
             __syncwarp();
         };
+        const uint32_t fill0 = fill;  // the first fill of this phase (the ring may hold descriptor chunks before)
         for (int i = i0; i < i1; ++i, ++fill) {
             const int st = fill % NSt;
             if (fill >= (uint32_t)NSt) {
                 if (lane == 0 && alive) alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
                 alive = __shfl_sync(0xffffffffu, alive, 0);
-                if (alive && touched(i - NSt)) {
+                if (alive && fill - NSt >= fill0 && touched(i - NSt)) {
                     bool ok = true;  // (complete: the consumers released it)
                     if (lane == 0) ok = mbar_wait(&full[st], ((fill / NSt) - 1) & 1, c.status);
                     if (__shfl_sync(0xffffffffu, ok, 0)) refresh(i - NSt, st);
@@ -840,7 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = max(i0, i1 - NSt); i < i1; ++i) {
             if (!alive || !touched(i)) continue;
-            const uint32_t f = (uint32_t)(i - i0);
+            const uint32_t f = fill0 + (uint32_t)(i - i0);
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&full[f % NSt], (f / NSt) & 1, c.status);
             if (__shfl_sync(0xffffffffu, ok, 0)) refresh(i, (int)(f % NSt));
@@ -1003,7 +1192,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     int ns = 6;
     const int fixed_bytes = 4 * (round4(pl.slice) * 2 + (p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0) +
                                  C * pl.gcap + 32 + 4 * pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
-    const int budget = 227 * 1024 - 1024 /*align*/ - 8 * 1024 /*static shared memory headroom*/;
+    const int budget = 227 * 1024 - 1024 /*align*/ - 10 * 1024 /*static shared memory headroom*/;
     while (ns > max(2, min_stages) && ns * stage + fixed_bytes + ns * (16 + (int)sizeof(StageInfo)) > budget) --ns;
     pl.n_stages = ns;
     off = ns * stage;
@@ -1096,9 +1285,11 @@ int active_clusters_any(const sba_cache& c, const sba_select_params& p, const Pl
 
 template <int kBlk, int kScorer, int kGM>
 int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaStream_t stream) {
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, td;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
     if (!make_kv_tmap(&tk, c.k, rows, kBlk) || !make_kv_tmap(&tv, c.v, rows, kBlk)) return SBA_ERR_CUDA;
+    if (!make_desc_tmap(&td, kScorer == SBA_SCORER_QUEST ? c.desc : (void*)c.kg, (uint64_t)c.num_pages, c.H_kv, kBlk))
+        return SBA_ERR_CUDA;
     cudaError_t e = prepare_kernel<kBlk, kScorer, kGM>(pl.smem);
     if (e != cudaSuccess) {
         note_cuda_error(e);
@@ -1124,7 +1315,7 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     a.sel_cap = pl.sel_cap;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = step_config(c, pl, stream, attr);
-    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM>, tk, tv, a);
+    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM>, tk, tv, td, a);
     if (e != cudaSuccess) {
         note_cuda_error(e);
         return SBA_ERR_CUDA;
