@@ -219,13 +219,13 @@ __device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t peer) 
 
 __device__ __forceinline__ uint32_t ld_peer_u32(uint32_t addr) {
     uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 
 __device__ __forceinline__ float ld_peer_f32(uint32_t addr) {
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
 }
 
@@ -234,7 +234,7 @@ __device__ __forceinline__ uint4 ld_peer_v4(uint32_t addr) {
     asm volatile("ld.shared::cluster.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(addr)
-                 : "memory");
+                 );
     return v;
 }
 

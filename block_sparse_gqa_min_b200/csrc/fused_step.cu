@@ -71,10 +71,8 @@ struct StepArgs {
     // shared-memory layout (bytes from the 1024-aligned base) and capacities
     int n_stages;
     int slice;      // largest slice: ceil(max_blocks / C) rounded up to a multiple of 4
-    int off_keys, off_pages, off_u, off_gmax, off_ckey, off_cidx, off_cpage, off_crank, off_sel, off_selp,
-        off_recv, off_bars;
-    int gcap;       // group maxima per CTA slot
-    int ccap;       // candidate slots (cluster total)
+    int off_keys, off_pages, off_u, off_crank, off_sel, off_selp, off_recv, off_bars;
+    int ccap;       // candidates ranked exactly (keys at or above the group-maxima bound)
     int sel_cap;    // words in sel / sel_page
 };
 
@@ -298,8 +296,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ __align__(16) float wgt_s[kMaxGroup][kCW];  // merge weights of the consumer warps
     __shared__ float lse_all[kMaxCluster * kMaxGroup];
     __shared__ float mz_all[kMaxCluster * kMaxGroup][2];
-    __shared__ int end_all[kMaxCluster];    // candidates each CTA pushed
-    __shared__ int pre_s[kMaxCluster + 1];  // their prefix
     __shared__ int local_page[kMaxLocal];
     __shared__ __align__(16) float pooled[3 * kHeadDim];     // refresh-before-score scratch
     __shared__ __align__(16) float pooled_b0[3 * kHeadDim];  // pushed pooled summary of B0
@@ -310,10 +306,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* keys = reinterpret_cast<uint32_t*>(dyn + a.off_keys);  // own slice
     int* pages = reinterpret_cast<int*>(dyn + a.off_pages);          // own slice
     float* u_s = reinterpret_cast<float*>(dyn + a.off_u);            // gate: [G][slice]
-    uint32_t* gmax_all = reinterpret_cast<uint32_t*>(dyn + a.off_gmax);  // [C][gcap]
-    uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + a.off_ckey);      // [ccap]
-    int* cidx = reinterpret_cast<int*>(dyn + a.off_cidx);
-    int* cpage = reinterpret_cast<int*>(dyn + a.off_cpage);
     int* crank = reinterpret_cast<int*>(dyn + a.off_crank);
     int* sel = reinterpret_cast<int*>(dyn + a.off_sel);
     int* sel_page = reinterpret_cast<int*>(dyn + a.off_selp);
@@ -502,7 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 } else {
                     // u = q . kg on tensor cores: tiles of 16 blocks (rows) x 8 heads (columns);
-                    // kg = hi + lo in tf32 (hi = kg rounded, lo = the rounded remainder); four
+                    // kg = hi + lo (hi = kg rounded to tf32, lo = the exact remainder, read by the MMA
+                    // truncated to tf32: about 21 bits of kg in all); four
                     // accumulators per tile (channel half x hi/lo) keep the MMA chains short, and
                     // a warp's tiles of the stage run interleaved when registers allow
                     constexpr int kTl = (kIt == 2 && NTq == 1) ? 2 : 1;
@@ -533,9 +526,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                         e ? x1.w : x1.y};
                                     uint32_t hi[4], lo[4];
 #pragma unroll
-                                    for (int u = 0; u < 4; ++u) {
+                                    for (int u = 0; u < 4; ++u) {  // (the MMA reads lo's top 19 bits)
                                         hi[u] = to_tf32(v[u]);
-                                        lo[u] = to_tf32(v[u] - __uint_as_float(hi[u]));
+                                        lo[u] = __float_as_uint(v[u] - __uint_as_float(hi[u]));
                                     }
                                     const int ah = (p >> 2) * 2;  // accumulator pair of this channel half
 #pragma unroll
@@ -713,65 +706,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncthreads();
     }
-    // group size: the largest power of two in [4, 128] leaving >= 2k groups
-    int gsh = 7;  // log2 of the group size
-    if (!trivial)
+    // every CTA's keys are final: each CTA pulls all keys of [0, NC) and selects on its own
+    if (app_e >= 0) fence_proxy_async_global();  // the appended rows, for the decode's tile loads
+    cluster_sync();
+    if (trivial) {
+        const int first = k <= 0 ? NC : 0;
+        for (int i = tid; i < N - first; i += kThreads) {
+            sel[i] = first + i;
+            sel_page[i] = first + i >= NC ? local_page[first + i - NC] : -1;
+        }
+    } else {
+        // all keys into the idle ring, 16 bytes at a time (a slice is a multiple of 4 blocks),
+        // four loads in flight per thread
+        uint32_t* kall = reinterpret_cast<uint32_t*>(dyn);
+        const int nv = (NC + 3) / 4;
+        for (int v0 = tid; v0 < nv; v0 += 4 * kThreads) {
+            uint4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + u * kThreads, j = 4 * v, p = j / slice;
+                if (v < nv)
+                    x[u] = p == r ? *reinterpret_cast<const uint4*>(keys + (j - j0))
+                                  : ld_peer_v4(peer_addr(keys + (j - p * slice), p));
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v = v0 + u * kThreads, j = 4 * v;
+                if (v < nv) {
+                    if (j + 1 >= NC) x[u].y = 0u;
+                    if (j + 2 >= NC) x[u].z = 0u;
+                    if (j + 3 >= NC) x[u].w = 0u;
+                    *reinterpret_cast<uint4*>(kall + j) = x[u];
+                }
+            }
+        }
+        // group size: the largest power of two in [4, 128] leaving >= 2k groups
+        int gsh = 7;
         while (gsh > 2 && ((NC + (1 << gsh) - 1) >> gsh) < 2 * k) --gsh;
-    const int gs = 1 << gsh;
-    // CTA p ranks the blocks [min(p*slice, NC), min(p*slice + slice, NC)) in groups of gs:
-    // every CTA knows every CTA's group count, hence where its maxima go
-    int goff = 0, ng_total = 0;
-    for (int p = 0; p < C; ++p) {
-        const int b0 = min(p * slice, NC);
-        const int ngp = (min(b0 + slice, NC) - b0 + gs - 1) >> gsh;
-        goff += p < r ? ngp : 0;
-        ng_total += ngp;
-    }
-    const int nown = jc1 - j0;  // my ranked candidates
-    if (tid == 0) misc[0] = -1;  // T0 (atomic minimum below)
-    // T0 below is a valid lower bound of the n-th score only when there are >= k groups
-    const bool bound = !trivial && ng_total >= k;
-    // the ranking below reads the maxima as 16-byte vectors: zeros (never larger) pad them
-    const int S_t0 = ng_total * 8 <= kThreads ? 8 : ng_total * 4 <= kThreads ? 4 : ng_total * 2 <= kThreads ? 2 : 1;
-    const int nvec_t0 = (ng_total + 4 * S_t0 - 1) / (4 * S_t0) * S_t0;
-    for (int i = ng_total + tid; i < 4 * nvec_t0; i += kThreads) gmax_all[i] = 0u;
-    if (bound) {
-        // maxima of my groups (four keys per thread, groups of gs/4 lanes), pushed to every CTA
-        const int lpg = gs / 4;
-        const uint4* kv = reinterpret_cast<const uint4*>(keys);
-        const int nv = (nown + 3) / 4;
+        const int gs = 1 << gsh, lpg = gs / 4;
+        const int ng = (NC + gs - 1) >> gsh;
+        // the rank counts below read 16-byte vectors: zeros (never larger) pad the group maxima
+        const int S0 = ng * 8 <= kThreads ? 8 : ng * 4 <= kThreads ? 4 : ng * 2 <= kThreads ? 2 : 1;
+        const int nv0 = (ng + 4 * S0 - 1) / (4 * S0) * S0;
+        uint32_t* gm = kall + ((NC + 127) & ~127);
+        uint32_t* ck = gm + ((4 * nv0 + 31) & ~31);
+        int* ci = reinterpret_cast<int*>(ck + a.ccap + 32);
+        for (int i = ng + tid; i < 4 * nv0; i += kThreads) gm[i] = 0u;
+        if (tid == 0) misc[0] = -1;  // T0 (atomic minimum below)
+        __syncthreads();
+        // group maxima (four keys per thread, groups of gs/4 lanes)
         for (int v0 = warp * 32; v0 < nv; v0 += kThreads) {
             const int v = v0 + lane;
             uint32_t m = 0;
             if (v < nv) {
-                const uint4 q = kv[v];
-                const int j = 4 * v;
-                m = max(max(j < nown ? q.x : 0u, j + 1 < nown ? q.y : 0u),
-                        max(j + 2 < nown ? q.z : 0u, j + 3 < nown ? q.w : 0u));
+                const uint4 q = *reinterpret_cast<const uint4*>(kall + 4 * v);
+                m = max(max(q.x, q.y), max(q.z, q.w));  // (keys past NC are zero)
             }
             for (int o = 1; o < lpg; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if ((lane & (lpg - 1)) == 0 && v < nv) {
-                uint32_t* dst = gmax_all + goff + v / lpg;
-                for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(dst, p), m);
-            }
+            if ((lane & (lpg - 1)) == 0 && v < nv) gm[v / lpg] = m;
         }
-    }
-    cluster_sync();  // every CTA's group maxima pushed
-    if (!trivial) {
+        __syncthreads();
+        // T0 = the k-th largest group maximum (k group maxima are k distinct blocks; with fewer
+        // than k groups T0 = 0).  Every thread counts, for one group maximum, the larger ones
+        // among a 1/S share of them.
         uint32_t T0 = 0;
-        if (bound) {
-            // T0 = the k-th largest group maximum (k group maxima are k distinct blocks).  Every
-            // thread counts, for one group maximum, the larger ones among a 1/S share of them.
-            const int S = S_t0;
-            const uint4* gv = reinterpret_cast<const uint4*>(gmax_all);
-            for (int t0 = 0; t0 < ng_total * S; t0 += kThreads) {
-                const int t = t0 + tid, g = t / S, sg = t % S;
+        if (ng >= k) {
+            const uint4* gv = reinterpret_cast<const uint4*>(gm);
+            for (int t0 = 0; t0 < ng * S0; t0 += kThreads) {
+                const int t = t0 + tid, g = t / S0, sg = t % S0;
                 int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
                 uint32_t x = 0;
-                if (g < ng_total) {
-                    x = gmax_all[g];
+                if (g < ng) {
+                    x = gm[g];
 #pragma unroll 4
-                    for (int v = sg; v < nvec_t0; v += S) {
+                    for (int v = sg; v < nv0; v += S0) {
                         const uint4 y = gv[v];
                         n0 += y.x > x;
                         n1 += y.y > x;
@@ -780,22 +788,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 int n = (n0 + n1) + (n2 + n3);
-                for (int o = 1; o < S; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-                uint32_t cand = (g < ng_total && n < k) ? x : 0xffffffffu;
+                for (int o = 1; o < S0; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+                uint32_t cand = (g < ng && n < k) ? x : 0xffffffffu;
                 cand = __reduce_min_sync(0xffffffffu, cand);
                 if (lane == 0 && cand != 0xffffffffu) atomicMin(reinterpret_cast<unsigned*>(&misc[0]), cand);
             }
             __syncthreads();
             T0 = (uint32_t)misc[0];
         }
-        // my candidates >= T0, in ascending block order, to my slots [r*cs, r*cs + cs) of every
-        // CTA's list (thread t takes a contiguous run of my keys), then their count (a count
-        // above cs marks an overflow)
-        const int cs = a.ccap / C;
-        const int per = (nown + kThreads - 1) / kThreads;
-        const int i0r = min(tid * per, nown), i1r = min(i0r + per, nown);
+        // the keys >= T0 in ascending block order: thread t scans a contiguous run of vectors (an
+        // odd number of them, so that a warp's 16-byte reads fall in distinct banks)
+        const uint4* kv = reinterpret_cast<const uint4*>(kall);
+        const int perv = ((nv + kThreads - 1) / kThreads) | 1;
+        const int v0r = min(tid * perv, nv), v1r = min(v0r + perv, nv);
         int cnt = 0;
-        for (int i = i0r; i < i1r; ++i) cnt += keys[i] >= T0;
+        for (int v = v0r; v < v1r; ++v) {
+            const uint4 q = kv[v];
+            const int j = 4 * v;
+            cnt += (q.x >= T0) + ((q.y >= T0) & (j + 1 < NC)) + ((q.z >= T0) & (j + 2 < NC)) +
+                   ((q.w >= T0) & (j + 3 < NC));
+        }
         int incl = cnt;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -804,76 +816,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 31) warp_tot[warp] = incl;
         __syncthreads();
-        int pos = incl - cnt, total = 0;
+        int pos = incl - cnt, m = 0;
         for (int w = 0; w < kThreads / 32; ++w) {
             const int x = warp_tot[w];
             pos += w < warp ? x : 0;
-            total += x;
+            m += x;
         }
-        for (int i = i0r; i < i1r && pos < cs; ++i) {
-            const uint32_t kk = keys[i];
-            if (kk < T0) continue;
-            const int slot = r * cs + pos;
-            const int pg = pages[i];
-            for (int p = 0; p < C; ++p) {
-                st_peer_u32(peer_addr(ckey + slot, p), kk);
-                st_peer_u32(peer_addr(cidx + slot, p), (uint32_t)(j0 + i));
-                st_peer_u32(peer_addr(cpage + slot, p), (uint32_t)pg);
-            }
-            ++pos;
-        }
-        if (tid < C) st_peer_u32(peer_addr(&end_all[r], tid), (uint32_t)total);
-    }
-    if (app_e >= 0) fence_proxy_async_global();  // the appended rows, for the decode's tile loads
-    cluster_sync();  // every candidate pushed
-    if (trivial) {
-        const int first = k <= 0 ? NC : 0;
-        for (int i = tid; i < N - first; i += kThreads) {
-            sel[i] = first + i;
-            sel_page[i] = first + i >= NC ? local_page[first + i - NC] : -1;
-        }
-    } else {
-        const int cs = a.ccap / C;
-        // prefix of the per-source counts, and whether a source overflowed
-        if (warp == 0) {
-            const int v = lane < C ? end_all[lane] : 0;
-            const bool ov = __any_sync(0xffffffffu, v > cs);
-            int incl = min(v, cs);
+        if (m <= a.ccap) {
+            for (int v = v0r; v < v1r; ++v) {
+                const uint4 q = kv[v];
+                const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+                for (int e = 0; e < 4; ++e)
+                    if (qs[e] >= T0 && 4 * v + e < NC) {
+                        ck[pos] = qs[e];
+                        ci[pos] = 4 * v + e;
+                        ++pos;
+                    }
             }
-            if (lane < C) pre_s[lane + 1] = incl;
-            if (lane == 0) {
-                pre_s[0] = 0;
-                misc[1] = ov;
-            }
-        }
-        __syncthreads();
-        const bool overflow = misc[1] != 0;
-        const int m = pre_s[C];
-        uint32_t* ck = reinterpret_cast<uint32_t*>(dyn);
-        int* ci = reinterpret_cast<int*>(ck + a.ccap + 32);
-        int* cp = ci + a.ccap + 32;
-        const int S = m * 8 <= kThreads ? 8 : m * 4 <= kThreads ? 4 : m * 2 <= kThreads ? 2 : 1;
-        const int nvec = (m + 4 * S - 1) / (4 * S) * S;  // 16-byte vectors of the ranking, padded
-        if (!overflow) {
-            // the per-source slots, compacted into [0, m) of the idle ring (ascending block order)
-            for (int i = tid; i < m; i += kThreads) {
-                int lo = 0, hi = C;  // the source p with pre_s[p] <= i < pre_s[p + 1]
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (pre_s[mid] <= i)
-                        lo = mid;
-                    else
-                        hi = mid;
-                }
-                const int slot = lo * cs + (i - pre_s[lo]);
-                ck[i] = ckey[slot];
-                ci[i] = cidx[slot];
-                cp[i] = cpage[slot];
-            }
+            const int S = m * 8 <= kThreads ? 8 : m * 4 <= kThreads ? 4 : m * 2 <= kThreads ? 2 : 1;
+            const int nvec = (m + 4 * S - 1) / (4 * S) * S;  // 16-byte vectors of the ranking, padded
             for (int i = m + tid; i < 4 * nvec; i += kThreads) {  // pads rank below everything
                 ck[i] = 0u;
                 ci[i] = 0x7fffffff;
@@ -916,35 +878,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     off += w < warp ? x : 0;
                     tot += x;
                 }
-                if (take) {
-                    const int p = off + __popc(bal & ((1u << lane) - 1u));
-                    sel[p] = ci[i];
-                    sel_page[p] = cp[i];
-                }
+                if (take) sel[off + __popc(bal & ((1u << lane) - 1u))] = ci[i];
                 run += tot;
                 __syncthreads();
             }
         } else {
-            // too many candidates (e.g. many equal scores): gather every score into the idle
-            // ring and run the exact selection there; pages come from the owning CTAs
-            uint32_t* kfull = reinterpret_cast<uint32_t*>(dyn);
-            uint32_t* gscr = kfull + ((NC + 3) & ~3);
+            // too many keys >= T0 (e.g. many equal scores): the exact selection on all keys
+            uint32_t* gscr = kall + ((NC + 3) & ~3);
             uint32_t* bkey = gscr + ((NC + 3) / 4 + 4);
             int* bidx = reinterpret_cast<int*>(bkey + 1024);
             int* brank = bidx + 1024;
-            for (int j = tid; j < NC; j += kThreads) {
-                const int p = j / slice;
-                kfull[j] = p == r ? keys[j - j0] : ld_peer_u32(peer_addr(keys + (j - p * slice), p));
-            }
             __syncthreads();
-            select_fast<kThreads>(kfull, NC, NC, k, sel, a.sel_cap, gscr, bkey, bidx, brank, 1024, misc + 2, hist,
+            select_fast<kThreads>(kall, NC, NC, k, sel, a.sel_cap, gscr, bkey, bidx, brank, 1024, misc + 2, hist,
                                   warp_tot, sh);
             __syncthreads();
-            for (int i = tid; i < k; i += kThreads) {
-                const int j = sel[i];
-                const int p = j / slice;
-                sel_page[i] = p == r ? pages[j - j0] : (int)ld_peer_u32(peer_addr(pages + (j - p * slice), p));
-            }
+        }
+        // pages of the selected blocks: from the slice owners (or computed, for a contiguous cache)
+        for (int i = tid; i < k; i += kThreads) {
+            const int j = sel[i];
+            const int p = j / slice;
+            sel_page[i] = c.block_table == nullptr ? page_quiet(c, s, j)
+                          : p == r                 ? pages[j - j0]
+                                                   : (int)ld_peer_u32(peer_addr(pages + (j - p * slice), p));
         }
         for (int i = tid; i < L; i += kThreads) {
             sel[k + i] = NC + i;
@@ -1164,9 +1119,8 @@ __global__ void fold_gate_kernel(const float* __restrict__ Wq, const float* __re
 }
 
 struct Plan {
-    int C, n_stages, smem, slice, gcap, ccap, sel_cap;
-    int off_keys, off_pages, off_u, off_gmax, off_ckey, off_cidx, off_cpage, off_crank, off_sel, off_selp, off_recv,
-        off_bars;
+    int C, n_stages, smem, slice, ccap, sel_cap;
+    int off_keys, off_pages, off_u, off_crank, off_sel, off_selp, off_recv, off_bars;
 };
 
 int round4(int x) { return (x + 3) & ~3; }
@@ -1177,7 +1131,6 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     const int G = c.H_q / c.H_kv;
     const int stage = c.b * kDescBytes;
     pl.slice = round4((c.max_blocks + C - 1) / C);
-    pl.gcap = round4((pl.slice + 3) / 4);
     pl.ccap = 1024;
     pl.sel_cap = round4(n_max_sel);
     const int E = G * kHeadDim;
@@ -1191,7 +1144,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + (c.b == 64 ? 1 : 0);
     int ns = 6;
     const int fixed_bytes = 4 * (round4(pl.slice) * 2 + (p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0) +
-                                 C * pl.gcap + 32 + 4 * pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
+                                 pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
     const int budget = 227 * 1024 - 1024 /*align*/ - 10 * 1024 /*static shared memory headroom*/;
     while (ns > max(2, min_stages) && ns * stage + fixed_bytes + ns * (16 + (int)sizeof(StageInfo)) > budget) --ns;
     pl.n_stages = ns;
@@ -1199,18 +1152,18 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     pl.off_keys = take(pl.slice);
     pl.off_pages = take(pl.slice);
     pl.off_u = take(p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0);
-    pl.off_gmax = take(C * pl.gcap + 32);
-    pl.off_ckey = take(pl.ccap);
-    pl.off_cidx = take(pl.ccap);
-    pl.off_cpage = take(pl.ccap);
     pl.off_crank = take(pl.ccap);
     pl.off_sel = take(pl.sel_cap);
     pl.off_selp = take(pl.sel_cap);
     pl.off_recv = take(C * ((E + C - 1) / C));
     pl.off_bars = off;
     pl.smem = pl.off_bars + ns * (16 + (int)sizeof(StageInfo)) + 1024;
-    // the fallback selection needs max_blocks + max_blocks/4 + 3*1024 words of the ring
-    if ((c.max_blocks + c.max_blocks / 4 + 8 + 3 * 1024) * 4 > ns * stage) pl.smem = 1 << 30;
+    // the selection keeps every key, the group maxima and the candidates (or the fallback's
+    // scratch) in the ring
+    const int mb128 = (c.max_blocks + 127) & ~127;
+    const int sel_words =
+        max(mb128 + c.max_blocks / 4 + 64 + 2 * (pl.ccap + 32), mb128 + c.max_blocks / 4 + 16 + 3 * 1024);
+    if (sel_words * 4 > ns * stage) pl.smem = 1 << 30;
     return pl;
 }
 
@@ -1301,16 +1254,11 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     a.off_keys = pl.off_keys;
     a.off_pages = pl.off_pages;
     a.off_u = pl.off_u;
-    a.off_gmax = pl.off_gmax;
-    a.off_ckey = pl.off_ckey;
-    a.off_cidx = pl.off_cidx;
-    a.off_cpage = pl.off_cpage;
     a.off_crank = pl.off_crank;
     a.off_sel = pl.off_sel;
     a.off_selp = pl.off_selp;
     a.off_recv = pl.off_recv;
     a.off_bars = pl.off_bars;
-    a.gcap = pl.gcap;
     a.ccap = pl.ccap;
     a.sel_cap = pl.sel_cap;
     cudaLaunchAttribute attr[2];
