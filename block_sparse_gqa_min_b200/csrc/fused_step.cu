@@ -261,11 +261,16 @@ __device__ __forceinline__ void refresh_from_stage(const sba_cache& c, const uin
 __device__ __forceinline__ void quest_coef(float (&coef)[8], const __nv_bfloat16* qg, int G, int lane) {
     const int ch0 = (lane & 15) * 8;
     const bool use_max = lane >= 16;
+    uint4 w[kMaxGroup];  // every head's load in flight at once
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g)
+        if (g < G) w[g] = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)g * kHeadDim + ch0));
 #pragma unroll
     for (int e = 0; e < 8; ++e) coef[e] = 0.f;
-    for (int g = 0; g < G; ++g) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qg + (int64_t)g * kHeadDim + ch0));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+        if (g >= G) break;
+        const uint32_t ws[4] = {w[g].x, w[g].y, w[g].z, w[g].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float x0 = bf16_lo(ws[e]), x1 = bf16_hi(ws[e]);
@@ -340,10 +345,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     pdl_wait();
     pdl_trigger();
+    const int len = __ldg(c.seq_lens + s);  // (both loads in flight while the work below is issued)
+    const int p0raw = a.n_new > 0 ? __ldg(a.pos_start + s) : 0;
+    // A contiguous cache's descriptors need no length to be located: the first ring stages of
+    // this CTA's slice (a fixed share of max_blocks) are requested before the lengths arrive.
+    const bool contiguous = c.block_table == nullptr;
+    const int nspec = contiguous ? min(NSt, (a.slice + kBlk - 1) / kBlk) : 0;
+    if (contiguous && warp == kProducer && lane == 0)
+        for (int f = 0; f < nspec; ++f) {
+            mbar_arrive_expect_tx(&full[f], TG::kStage);
+            tma_load_4d(dyn + (size_t)f * TG::kStage, &tmD, &full[f], 0, 0, h, s * mb + r * a.slice + f * kBlk);
+        }
+
+    // ... nor do the query-side scoring coefficients of the consumer warps (ring scoring)
+    constexpr int NTq = kGM > 8 ? 2 : 1;  // gate: 8-head n-tiles
+    float coef[8];
+    uint32_t qf[NTq][8][4];
+    if (contiguous && warp < kCW) {
+        if (kScorer == SBA_SCORER_QUEST) {
+            quest_coef(coef, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
+        } else {
+            // B fragments: head nt*8 + lane/4, channels 16p + 4(lane%4) + 0..3 (bf16 is exact in tf32)
+#pragma unroll
+            for (int nt = 0; nt < NTq; ++nt) {
+                const int head = nt * 8 + (lane >> 2);
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    uint2 w = make_uint2(0u, 0u);
+                    if (head < G)
+                        w = __ldg(reinterpret_cast<const uint2*>(a.q + ((int64_t)s * c.H_q + h * G + head) * kHeadDim +
+                                                                16 * p + 4 * (lane & 3)));
+                    qf[nt][p][0] = w.x << 16;
+                    qf[nt][p][1] = w.x & 0xffff0000u;
+                    qf[nt][p][2] = w.y << 16;
+                    qf[nt][p][3] = w.y & 0xffff0000u;
+                }
+            }
+        }
+    }
 
     // ---------------- shapes of this (sequence, group) ----------------
-    const int len = __ldg(c.seq_lens + s);
-    const int p0raw = a.n_new > 0 ? __ldg(a.pos_start + s) : 0;
     int N = blocks_of(len, kBlk);
     if (N > mb) {
         if (tid == 0 && r == 0) report(c.status, SBA_DEV_BAD_POSITION);
@@ -354,7 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int NC = N - L;                                               // ranked candidates [0, NC)
     const int NSc = kScorer == SBA_SCORER_GATE ? max(N - 1, 0) : NC;   // blocks this step scores
     // this sequence's scored blocks [0, NSc) in C equal slices (sequences differ in length)
-    const int slice = min(max(4, ((NSc + C - 1) / C + 3) & ~3), a.slice);
+    // (a contiguous cache keeps the fixed slices its early loads assumed)
+    const int slice = contiguous ? a.slice : min(max(4, ((NSc + C - 1) / C + 3) & ~3), a.slice);
     const int j0 = min(r * slice, NSc), js1 = min(j0 + slice, NSc);    // my scored blocks [j0, js1)
     const int jc1 = max(j0, min(js1, NC));                              // my ranked candidates [j0, jc1)
     for (int j = j0 + tid; j < js1; j += kThreads) {
@@ -412,50 +454,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a ring stage (128-byte quarter rows, 128-byte swizzle); the two consumer groups take
         // alternate stages, each warp 16 descriptors (one tensor-core tile for the gate) per
         // 64 of the stage.
+        // Fills [0, nspec) were requested early.  Normally they are chunks 0.. of the slice (those
+        // past its end are drained unread); after a refresh before scoring their contents may
+        // be stale, so they are drained and every chunk is requested again.
         const int nch = (js1 - j0 + kBlk - 1) / kBlk;
+        const int skip = touched_scored ? nspec : 0;
+        const int ntot = touched_scored ? nspec + nch : max(nch, nspec);
         if (warp == kProducer) {
             if (lane == 0) {
                 bool alive = true;
-                for (int f = 0; f < nch && alive; ++f) {
+                for (int f = nspec; f < ntot && alive; ++f) {
                     const int st = f % NSt;
                     if (f >= NSt) alive = mbar_wait(&empty[st], ((f / NSt) - 1) & 1, c.status);
                     if (alive) {
                         mbar_arrive_expect_tx(&full[st], TG::kStage);
-                        tma_load_4d(dyn + (size_t)st * TG::kStage, &tmD, &full[st], 0, 0, h, s * mb + j0 + f * kBlk);
+                        tma_load_4d(dyn + (size_t)st * TG::kStage, &tmD, &full[st], 0, 0, h,
+                                    s * mb + j0 + (f - skip) * kBlk);
                     }
                 }
             }
         } else {
             const int grp = warp / kGW, gw = warp % kGW;
             constexpr int kIt = kBlk / 64;         // 16-descriptor pieces of a stage per warp
-            constexpr int NTq = kGM > 8 ? 2 : 1;  // gate: 8-head n-tiles
-            float coef[8];
-            uint32_t qf[NTq][8][4];
-            if (kScorer == SBA_SCORER_QUEST) {
-                quest_coef(coef, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
-            } else {
-                // B fragments: head nt*8 + lane/4, channels 16p + 4(lane%4) + 0..3 (bf16 is exact in tf32)
-#pragma unroll
-                for (int nt = 0; nt < NTq; ++nt) {
-                    const int head = nt * 8 + (lane >> 2);
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        uint2 w = make_uint2(0u, 0u);
-                        if (head < G)
-                            w = __ldg(reinterpret_cast<const uint2*>(a.q + ((int64_t)s * c.H_q + h * G + head) * kHeadDim +
-                                                                    16 * p + 4 * (lane & 3)));
-                        qf[nt][p][0] = w.x << 16;
-                        qf[nt][p][1] = w.x & 0xffff0000u;
-                        qf[nt][p][2] = w.y << 16;
-                        qf[nt][p][3] = w.y & 0xffff0000u;
-                    }
-                }
-            }
             bool alive = true;
-            for (int f = grp; f < nch; f += kGroups) {
+            for (int f = grp; f < ntot; f += kGroups) {
                 const int st = f % NSt;
                 if (alive) alive = mbar_wait(&full[st], (f / NSt) & 1, c.status);
-                const int cb = j0 + f * kBlk, nblk = min(kBlk, js1 - cb);
+                const int cb = j0 + (f - skip) * kBlk;
+                const int nblk = f < skip ? 0 : min(kBlk, js1 - cb);  // (<= 0: a drained fill)
                 const uint8_t* stage = dyn + (size_t)st * TG::kStage;
                 if (kScorer == SBA_SCORER_QUEST) {
 #pragma unroll
@@ -566,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
         }
-        fill = (uint32_t)nch;
+        fill = (uint32_t)ntot;
     } else {
     // Paged cache: every warp streams descriptors straight into registers: kRB blocks per
     // warp and round, lane l holding bytes [16 l, 16 l + 16) of each 512-byte descriptor;
@@ -740,9 +766,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        // group size: the largest power of two in [4, 128] leaving >= 2k groups
+        // group size: the largest power of two in [4, 128] leaving >= 5k/4 groups (T0 costs ~ng^2
+        // comparisons, the exact rank ~m^2 for the m keys >= T0; this balances the two for
+        // random scores: e.g. 2044 blocks, k = 99 -> 128 groups of 16, m ~ 185)
         int gsh = 7;
-        while (gsh > 2 && ((NC + (1 << gsh) - 1) >> gsh) < 2 * k) --gsh;
+        while (gsh > 2 && ((NC + (1 << gsh) - 1) >> gsh) * 4 < 5 * k) --gsh;
         const int gs = 1 << gsh, lpg = gs / 4;
         const int ng = (NC + gs - 1) >> gsh;
         // the rank counts below read 16-byte vectors: zeros (never larger) pad the group maxima
