@@ -71,7 +71,7 @@ struct StepArgs {
     // shared-memory layout (bytes from the 1024-aligned base) and capacities
     int n_stages;
     int slice;      // largest slice: ceil(max_blocks / C) rounded up to a multiple of 4
-    int off_keys, off_pages, off_u, off_crank, off_sel, off_selp, off_recv, off_bars;
+    int off_keys, off_pages, off_u, off_kall, off_gm, off_crank, off_sel, off_selp, off_recv, off_bars;
     int ccap;       // candidates ranked exactly (keys at or above the group-maxima bound)
     int sel_cap;    // words in sel / sel_page
 };
@@ -406,6 +406,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int k = n_sel - L;
     const bool trivial = k <= 0 || k >= NC;  // take none / all of the candidates
+    // Selection geometry, known before scoring.  Every CTA receives every key (kall) and every
+    // CTA's group maxima (gmx: groups of gs blocks aligned to each slice) while the keys are
+    // produced, so that one cluster barrier later each CTA selects on its own.  The group size
+    // is the largest power of two in [4, 128] leaving >= 2k groups (T0 below costs ~ng^2
+    // comparisons, the exact rank ~m^2 for the m keys >= T0; more groups give a tighter T0).
+    int gsh = 7;
+    if (!trivial)
+        while (gsh > 2 && ((NC + (1 << gsh) - 1) >> gsh) < 2 * k) --gsh;
+    const int gs = 1 << gsh;
+    int goff = 0, ng = 0;
+    for (int p = 0; p < C; ++p) {
+        const int b0 = min(p * slice, NC);
+        const int ngp = (min(b0 + slice, NC) - b0 + gs - 1) >> gsh;
+        goff += p < r ? ngp : 0;
+        ng += ngp;
+    }
+    // (the gate's keys are produced after scoring, when the ring is idle everywhere)
+    uint32_t* kall = kScorer == SBA_SCORER_GATE ? reinterpret_cast<uint32_t*>(dyn)
+                                                : reinterpret_cast<uint32_t*>(dyn + a.off_kall);
+    uint32_t* gmx = reinterpret_cast<uint32_t*>(dyn + a.off_gm);
     for (int i = tid; i < L && i < kMaxLocal; i += kThreads) local_page[i] = page_quiet(c, s, NC + i);
 
     int n_new = a.n_new, p0 = 0, tb0 = 1, tb1 = 0;
@@ -514,7 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int i = n0 + 8 * rd + rs_block<8>(lane);
                             if ((lane & 3) == 0 && i < nblk) {
                                 const int jl = cb + i - j0;
-                                keys[jl] = pages[jl] >= 0 ? orderable_key(tot[rd][0]) : 0u;
+                                const uint32_t key = pages[jl] >= 0 ? orderable_key(tot[rd][0]) : 0u;
+                                keys[jl] = key;
+                                if (!trivial)
+                                    for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(kall + j0 + jl, p), key);
                             }
                         }
                     }
@@ -653,7 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float tot[1];
                 reduce_scatter<kRB, 1>(part, tot, lane);
                 const int j = base + rs_block<kRB>(lane);
-                if ((lane & 3) == 0 && j < js1) keys[j - j0] = pages[j - j0] >= 0 ? orderable_key(tot[0]) : 0u;
+                if ((lane & 3) == 0 && j < js1) {
+                    const uint32_t key = pages[j - j0] >= 0 ? orderable_key(tot[0]) : 0u;
+                    keys[j - j0] = key;
+                    if (!trivial)
+                        for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(kall + j, p), key);
+                }
             } else {
 #pragma unroll
                 for (int q4 = 0; q4 < kRB; q4 += 4) {
@@ -724,15 +752,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             lse_s[tid] = M > -INFINITY ? M + logf(Z) : -INFINITY;
         }
         __syncthreads();
-        // group score of my ranked blocks: sum over the group of g = exp(u - LSE)
-        for (int j = j0 + tid; j < jc1; j += kThreads) {
-            float sc = 0.f;
-            for (int g = 0; g < G; ++g) sc += expf(u_s[g * ustride + (j - j0)] - lse_s[g]);
-            keys[j - j0] = pages[j - j0] >= 0 ? orderable_key(sc) : 0u;
+        // group score of my ranked blocks: sum over the group of g = exp(u - LSE), four blocks per
+        // thread, pushed to every CTA
+        for (int v = tid; 4 * v < jc1 - j0; v += kThreads) {
+            const int jl = 4 * v;
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int g = 0; g < G; ++g) {
+                const float4 u4 = *reinterpret_cast<const float4*>(u_s + g * ustride + jl);
+                sc[0] += expf(u4.x - lse_s[g]);
+                sc[1] += expf(u4.y - lse_s[g]);
+                sc[2] += expf(u4.z - lse_s[g]);
+                sc[3] += expf(u4.w - lse_s[g]);
+            }
+            uint32_t kk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                kk[e] = (jl + e < jc1 - j0 && pages[jl + e] >= 0) ? orderable_key(sc[e]) : 0u;
+            const uint4 k4 = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+            *reinterpret_cast<uint4*>(keys + jl) = k4;
+            if (!trivial)
+                for (int p = 0; p < C; ++p) st_peer_v4(peer_addr(kall + j0 + jl, p), k4);
         }
         __syncthreads();
     }
-    // every CTA's keys are final: each CTA pulls all keys of [0, NC) and selects on its own
+    // my keys are final: the maxima of my slice's groups go to every CTA (four keys per thread,
+    // groups of gs/4 lanes); zeros (never larger) pad the vectors the rank counts read
+    const int S0 = ng * 8 <= kThreads ? 8 : ng * 4 <= kThreads ? 4 : ng * 2 <= kThreads ? 2 : 1;
+    const int nv0 = (ng + 4 * S0 - 1) / (4 * S0) * S0;
+    if (!trivial) {
+        const int nown = jc1 - j0, lpg = gs / 4;
+        const uint4* kv = reinterpret_cast<const uint4*>(keys);
+        const int nvo = (nown + 3) / 4;
+        for (int v0 = warp * 32; v0 < nvo; v0 += kThreads) {
+            const int v = v0 + lane;
+            uint32_t m = 0;
+            if (v < nvo) {
+                const uint4 q = kv[v];
+                const int j = 4 * v;
+                m = max(max(j < nown ? q.x : 0u, j + 1 < nown ? q.y : 0u),
+                        max(j + 2 < nown ? q.z : 0u, j + 3 < nown ? q.w : 0u));
+            }
+            for (int o = 1; o < lpg; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((lane & (lpg - 1)) == 0 && v < nvo)
+                for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(gmx + goff + v / lpg, p), m);
+        }
+        for (int i = ng + tid; i < 4 * nv0; i += kThreads) gmx[i] = 0u;
+        if (tid == 0) misc[0] = -1;  // T0 (atomic minimum below)
+    }
+    // every CTA's keys and group maxima are in every CTA: each selects on its own
     if (app_e >= 0) fence_proxy_async_global();  // the appended rows, for the decode's tile loads
     cluster_sync();
     if (trivial) {
@@ -742,58 +809,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             sel_page[i] = first + i >= NC ? local_page[first + i - NC] : -1;
         }
     } else {
-        // all keys into the idle ring, 16 bytes at a time (a slice is a multiple of 4 blocks),
-        // four loads in flight per thread
-        uint32_t* kall = reinterpret_cast<uint32_t*>(dyn);
         const int nv = (NC + 3) / 4;
-        for (int v0 = tid; v0 < nv; v0 += 4 * kThreads) {
-            uint4 x[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int v = v0 + u * kThreads, j = 4 * v, p = j / slice;
-                if (v < nv)
-                    x[u] = p == r ? *reinterpret_cast<const uint4*>(keys + (j - j0))
-                                  : ld_peer_v4(peer_addr(keys + (j - p * slice), p));
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int v = v0 + u * kThreads, j = 4 * v;
-                if (v < nv) {
-                    if (j + 1 >= NC) x[u].y = 0u;
-                    if (j + 2 >= NC) x[u].z = 0u;
-                    if (j + 3 >= NC) x[u].w = 0u;
-                    *reinterpret_cast<uint4*>(kall + j) = x[u];
-                }
-            }
-        }
-        // group size: the largest power of two in [4, 128] leaving >= 5k/4 groups (T0 costs ~ng^2
-        // comparisons, the exact rank ~m^2 for the m keys >= T0; this balances the two for
-        // random scores: e.g. 2044 blocks, k = 99 -> 128 groups of 16, m ~ 185)
-        int gsh = 7;
-        while (gsh > 2 && ((NC + (1 << gsh) - 1) >> gsh) * 4 < 5 * k) --gsh;
-        const int gs = 1 << gsh, lpg = gs / 4;
-        const int ng = (NC + gs - 1) >> gsh;
-        // the rank counts below read 16-byte vectors: zeros (never larger) pad the group maxima
-        const int S0 = ng * 8 <= kThreads ? 8 : ng * 4 <= kThreads ? 4 : ng * 2 <= kThreads ? 2 : 1;
-        const int nv0 = (ng + 4 * S0 - 1) / (4 * S0) * S0;
-        uint32_t* gm = kall + ((NC + 127) & ~127);
-        uint32_t* ck = gm + ((4 * nv0 + 31) & ~31);
+        uint32_t* gm = gmx;
+        // candidates (and the fallback's scratch) in the idle ring, after the gate's keys
+        uint32_t* scr = kScorer == SBA_SCORER_GATE ? kall + ((NC + 127) & ~127) : reinterpret_cast<uint32_t*>(dyn);
+        uint32_t* ck = scr;
         int* ci = reinterpret_cast<int*>(ck + a.ccap + 32);
-        for (int i = ng + tid; i < 4 * nv0; i += kThreads) gm[i] = 0u;
-        if (tid == 0) misc[0] = -1;  // T0 (atomic minimum below)
-        __syncthreads();
-        // group maxima (four keys per thread, groups of gs/4 lanes)
-        for (int v0 = warp * 32; v0 < nv; v0 += kThreads) {
-            const int v = v0 + lane;
-            uint32_t m = 0;
-            if (v < nv) {
-                const uint4 q = *reinterpret_cast<const uint4*>(kall + 4 * v);
-                m = max(max(q.x, q.y), max(q.z, q.w));  // (keys past NC are zero)
-            }
-            for (int o = 1; o < lpg; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if ((lane & (lpg - 1)) == 0 && v < nv) gm[v / lpg] = m;
-        }
-        __syncthreads();
         // T0 = the k-th largest group maximum (k group maxima are k distinct blocks; with fewer
         // than k groups T0 = 0).  Every thread counts, for one group maximum, the larger ones
         // among a 1/S share of them.
@@ -912,7 +933,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else {
             // too many keys >= T0 (e.g. many equal scores): the exact selection on all keys
-            uint32_t* gscr = kall + ((NC + 3) & ~3);
+            uint32_t* gscr = scr;
             uint32_t* bkey = gscr + ((NC + 3) / 4 + 4);
             int* bidx = reinterpret_cast<int*>(bkey + 1024);
             int* brank = bidx + 1024;
@@ -1148,7 +1169,7 @@ __global__ void fold_gate_kernel(const float* __restrict__ Wq, const float* __re
 
 struct Plan {
     int C, n_stages, smem, slice, ccap, sel_cap;
-    int off_keys, off_pages, off_u, off_crank, off_sel, off_selp, off_recv, off_bars;
+    int off_keys, off_pages, off_u, off_kall, off_gm, off_crank, off_sel, off_selp, off_recv, off_bars;
 };
 
 int round4(int x) { return (x + 3) & ~3; }
@@ -1171,8 +1192,11 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     // the ring comes first (1024-aligned); the fallback selection reuses it
     const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + (c.b == 64 ? 1 : 0);
     int ns = 6;
-    const int fixed_bytes = 4 * (round4(pl.slice) * 2 + (p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0) +
-                                 pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
+    const int mb128 = (c.max_blocks + 127) & ~127;
+    const int kall_words = p.scorer == SBA_SCORER_GATE ? 0 : mb128 + 4;  // (the gate's keys use the ring)
+    const int gm_words = C * round4((pl.slice + 3) / 4) + 64;
+    const int fixed_bytes = 4 * (round4(pl.slice) * 2 + (p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0) + kall_words +
+                                 gm_words + pl.ccap + 2 * pl.sel_cap + round4(C * ((E + C - 1) / C)) + 64);
     const int budget = 227 * 1024 - 1024 /*align*/ - 10 * 1024 /*static shared memory headroom*/;
     while (ns > max(2, min_stages) && ns * stage + fixed_bytes + ns * (16 + (int)sizeof(StageInfo)) > budget) --ns;
     pl.n_stages = ns;
@@ -1180,17 +1204,18 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     pl.off_keys = take(pl.slice);
     pl.off_pages = take(pl.slice);
     pl.off_u = take(p.scorer == SBA_SCORER_GATE ? G * pl.slice : 0);
+    pl.off_kall = take(kall_words);
+    pl.off_gm = take(gm_words);
     pl.off_crank = take(pl.ccap);
     pl.off_sel = take(pl.sel_cap);
     pl.off_selp = take(pl.sel_cap);
     pl.off_recv = take(C * ((E + C - 1) / C));
     pl.off_bars = off;
     pl.smem = pl.off_bars + ns * (16 + (int)sizeof(StageInfo)) + 1024;
-    // the selection keeps every key, the group maxima and the candidates (or the fallback's
-    // scratch) in the ring
-    const int mb128 = (c.max_blocks + 127) & ~127;
-    const int sel_words =
-        max(mb128 + c.max_blocks / 4 + 64 + 2 * (pl.ccap + 32), mb128 + c.max_blocks / 4 + 16 + 3 * 1024);
+    // the selection keeps the candidates (or the fallback's scratch) in the ring, after the
+    // gate's keys
+    const int sel_words = (p.scorer == SBA_SCORER_GATE ? mb128 : 0) +
+                          max(2 * (pl.ccap + 32), c.max_blocks / 4 + 16 + 3 * 1024);
     if (sel_words * 4 > ns * stage) pl.smem = 1 << 30;
     return pl;
 }
@@ -1282,6 +1307,8 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     a.off_keys = pl.off_keys;
     a.off_pages = pl.off_pages;
     a.off_u = pl.off_u;
+    a.off_kall = pl.off_kall;
+    a.off_gm = pl.off_gm;
     a.off_crank = pl.off_crank;
     a.off_sel = pl.off_sel;
     a.off_selp = pl.off_selp;
