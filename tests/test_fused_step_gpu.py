@@ -86,6 +86,9 @@ FUSED_CASES = [
     dict(H_q=4, H_kv=4, b=64, len_lo=1, len_hi=1, n_budget=4, n_local=1),            # one token
     dict(H_q=8, H_kv=8, b=128, len_lo=1000, len_hi=1000, n_budget=100, n_local=2),  # select all
     dict(H_q=6, H_kv=3, b=64, len_lo=64, len_hi=5000, B=5, n_budget=3, n_local=1, paged=True),
+    # contiguous pages, lengths that differ: slices are fixed shares of max_blocks, so the CTAs
+    # past a short sequence's end drain their early descriptor loads unread
+    dict(H_q=8, H_kv=2, b=64, len_lo=100, len_hi=6000, B=4, n_budget=8, n_local=2),
 ]
 
 
@@ -116,6 +119,7 @@ FUSED_GATE_CASES = [
     dict(H_q=10, H_kv=2, b=64, len_lo=3000, len_hi=7000, B=2, n_budget=6, n_local=2, paged=True),
     dict(H_q=5, H_kv=1, b=64, len_lo=65, len_hi=65, n_budget=4, n_local=2),          # C = 1 historical
     dict(H_q=8, H_kv=4, b=128, len_lo=200, len_hi=5000, B=3, n_budget=5, n_local=0, paged=True),
+    dict(H_q=10, H_kv=2, b=64, len_lo=300, len_hi=6000, B=3, n_budget=6, n_local=2),  # contiguous, lengths differ
 ]
 
 
