@@ -187,54 +187,69 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Descriptor of a touched block from its K tile staged in shared memory, by one warp:
-// lane = 16-byte chunk (8 channels) of a row x token parity.  Quest: the min/max rows
-// (exact in bf16) go to the cache; gate: the pooled [max | min | avg] summary is pushed
-// to every CTA of the cluster, which project it after the merge.
-template <int kBlk, int kScorer>
-__device__ __forceinline__ void refresh_from_stage(const sba_cache& c, const uint8_t* stage, int valid, int64_t pg,
-                                                   int h, float* pooled_b0, int C, int lane) {
-    using TG = TileGeom<kBlk>;
-    const int ck = lane & 15, cc = ck & 7;
-    const uint8_t* kt = stage + (ck >> 3) * TG::kHalf;
+// Descriptor of a touched block from its K rows staged in shared memory (one or two 64-row
+// stages), by one warp: lane = 16-byte chunk (8 channels) of a row x token parity.  The min,
+// max (exact in bf16) and, for the gate, the fp32 sum accumulate over the stages.
+struct RefreshAcc {
     uint32_t mn[4], mx[4];
     float sm[8];
+};
+
+__device__ __forceinline__ void refresh_init(RefreshAcc& acc) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        mn[e] = 0x7f807f80u;  // +inf, +inf
-        mx[e] = 0xff80ff80u;  // -inf, -inf
-        sm[2 * e] = sm[2 * e + 1] = 0.f;
+        acc.mn[e] = 0x7f807f80u;  // +inf, +inf
+        acc.mx[e] = 0xff80ff80u;  // -inf, -inf
+        acc.sm[2 * e] = acc.sm[2 * e + 1] = 0.f;
     }
+}
+
+template <int kScorer>
+__device__ __forceinline__ void refresh_accum(RefreshAcc& acc, const uint8_t* stage, int valid, int lane) {
+    using TG = TileGeom<64>;
+    const int ck = lane & 15, cc = ck & 7;
+    const uint8_t* kt = stage + (ck >> 3) * TG::kHalf;
 #pragma unroll 4
     for (int t = lane >> 4; t < valid; t += 2) {
         const uint4 w = *reinterpret_cast<const uint4*>(kt + t * 128 + ((cc ^ (t & 7)) << 4));
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            mn[e] = bf16x2_min(mn[e], ws[e]);
-            mx[e] = bf16x2_max(mx[e], ws[e]);
+            acc.mn[e] = bf16x2_min(acc.mn[e], ws[e]);
+            acc.mx[e] = bf16x2_max(acc.mx[e], ws[e]);
             if (kScorer == SBA_SCORER_GATE) {
-                sm[2 * e] += bf16_lo(ws[e]);
-                sm[2 * e + 1] += bf16_hi(ws[e]);
+                acc.sm[2 * e] += bf16_lo(ws[e]);
+                acc.sm[2 * e + 1] += bf16_hi(ws[e]);
             }
         }
     }
+}
+
+// Quest: the min/max rows go to the cache; gate: the pooled [max | min | avg] summary is
+// pushed to every CTA of the cluster, which project it after the merge.
+template <int kScorer>
+__device__ __forceinline__ void refresh_finish(const sba_cache& c, RefreshAcc& acc, int valid, int64_t pg, int h,
+                                               float* pooled_b0, int C, int lane) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {  // the other token parity
-        mn[e] = bf16x2_min(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], 16));
-        mx[e] = bf16x2_max(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
+        acc.mn[e] = bf16x2_min(acc.mn[e], __shfl_xor_sync(0xffffffffu, acc.mn[e], 16));
+        acc.mx[e] = bf16x2_max(acc.mx[e], __shfl_xor_sync(0xffffffffu, acc.mx[e], 16));
         if (kScorer == SBA_SCORER_GATE) {
-            sm[2 * e] += __shfl_xor_sync(0xffffffffu, sm[2 * e], 16);
-            sm[2 * e + 1] += __shfl_xor_sync(0xffffffffu, sm[2 * e + 1], 16);
+            acc.sm[2 * e] += __shfl_xor_sync(0xffffffffu, acc.sm[2 * e], 16);
+            acc.sm[2 * e + 1] += __shfl_xor_sync(0xffffffffu, acc.sm[2 * e + 1], 16);
         }
     }
     if (lane >= 16) return;
+    const int ck = lane;
     if (kScorer == SBA_SCORER_QUEST) {
         uint8_t* d = reinterpret_cast<uint8_t*>(c.desc) + (pg * c.H_kv + h) * 2 * kHeadDim * 2;
-        *reinterpret_cast<uint4*>(d + ck * 16) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
-        *reinterpret_cast<uint4*>(d + 2 * kHeadDim + ck * 16) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
+        *reinterpret_cast<uint4*>(d + ck * 16) = make_uint4(acc.mn[0], acc.mn[1], acc.mn[2], acc.mn[3]);
+        *reinterpret_cast<uint4*>(d + 2 * kHeadDim + ck * 16) = make_uint4(acc.mx[0], acc.mx[1], acc.mx[2], acc.mx[3]);
     } else {
         const float inv = 1.f / (float)valid;
+        const uint32_t* mx = acc.mx;
+        const uint32_t* mn = acc.mn;
+        const float* sm = acc.sm;
         const float4 hi0 = make_float4(bf16_lo(mx[0]), bf16_hi(mx[0]), bf16_lo(mx[1]), bf16_hi(mx[1]));
         const float4 hi1 = make_float4(bf16_lo(mx[2]), bf16_hi(mx[2]), bf16_lo(mx[3]), bf16_hi(mx[3]));
         const float4 lo0 = make_float4(bf16_lo(mn[0]), bf16_hi(mn[0]), bf16_lo(mn[1]), bf16_hi(mn[1]));
@@ -291,7 +306,11 @@ template <int kBlk, int kScorer, int kGM>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmD, StepArgs a) {
-    using TG = TileGeom<kBlk>;
+    // The ring holds 64-token stages (32 KB): a block of 128 tokens takes two consecutive fills,
+    // and a descriptor chunk is 64 descriptors.
+    using TG = TileGeom<64>;
+    constexpr int kSub = kBlk / 64;   // ring fills per block
+    constexpr int kSC = 64;           // descriptors per scoring fill
     constexpr int kMaxLocal = 64;
     __shared__ uint32_t hist[256];
     __shared__ int warp_tot[kThreads / 32];
@@ -350,11 +369,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // A contiguous cache's descriptors need no length to be located: the first ring stages of
     // this CTA's slice (a fixed share of max_blocks) are requested before the lengths arrive.
     const bool contiguous = c.block_table == nullptr;
-    const int nspec = contiguous ? min(NSt, (a.slice + kBlk - 1) / kBlk) : 0;
+    const int nspec = contiguous ? min(NSt, (a.slice + kSC - 1) / kSC) : 0;
     if (contiguous && warp == kProducer && lane == 0)
         for (int f = 0; f < nspec; ++f) {
             mbar_arrive_expect_tx(&full[f], TG::kStage);
-            tma_load_4d(dyn + (size_t)f * TG::kStage, &tmD, &full[f], 0, 0, h, s * mb + r * a.slice + f * kBlk);
+            tma_load_4d(dyn + (size_t)f * TG::kStage, &tmD, &full[f], 0, 0, h, s * mb + r * a.slice + f * kSC);
         }
 
     // ... nor do the query-side scoring coefficients of the consumer warps (ring scoring)
@@ -477,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Fills [0, nspec) were requested early.  Normally they are chunks 0.. of the slice (those
         // past its end are drained unread); after a refresh before scoring their contents may
         // be stale, so they are drained and every chunk is requested again.
-        const int nch = (js1 - j0 + kBlk - 1) / kBlk;
+        const int nch = (js1 - j0 + kSC - 1) / kSC;
         const int skip = touched_scored ? nspec : 0;
         const int ntot = touched_scored ? nspec + nch : max(nch, nspec);
         if (warp == kProducer) {
@@ -489,19 +508,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (alive) {
                         mbar_arrive_expect_tx(&full[st], TG::kStage);
                         tma_load_4d(dyn + (size_t)st * TG::kStage, &tmD, &full[st], 0, 0, h,
-                                    s * mb + j0 + (f - skip) * kBlk);
+                                    s * mb + j0 + (f - skip) * kSC);
                     }
                 }
             }
         } else {
             const int grp = warp / kGW, gw = warp % kGW;
-            constexpr int kIt = kBlk / 64;         // 16-descriptor pieces of a stage per warp
+            constexpr int kIt = kSC / 64;          // 16-descriptor pieces of a stage per warp
             bool alive = true;
             for (int f = grp; f < ntot; f += kGroups) {
                 const int st = f % NSt;
                 if (alive) alive = mbar_wait(&full[st], (f / NSt) & 1, c.status);
-                const int cb = j0 + (f - skip) * kBlk;
-                const int nblk = f < skip ? 0 : min(kBlk, js1 - cb);  // (<= 0: a drained fill)
+                const int cb = j0 + (f - skip) * kSC;
+                const int nblk = f < skip ? 0 : min(kSC, js1 - cb);  // (<= 0: a drained fill)
                 const uint8_t* stage = dyn + (size_t)st * TG::kStage;
                 if (kScorer == SBA_SCORER_QUEST) {
 #pragma unroll
@@ -980,63 +999,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         bool alive = true;
-        // blocks touched by this step's append get their descriptors from the staged K tiles
-        // here, before their stage is reused or, for the last NSt positions, after the loop
+        // Blocks touched by this step's append get their descriptors from their staged K rows,
+        // here: when the stage of a touched block's first fill is about to be reused (its other
+        // fill, issued after it, is then waited for), or, for the last fills, after the loop.
         auto touched = [&](int i) {
             const int j = sel[i];
             return tile_refresh && j >= tb0 && j <= tb1 && sel_page[i] >= 0;
         };
-        auto refresh = [&](int i, int st) {
-            const int j = sel[i];
-            refresh_from_stage<kBlk, kScorer>(c, dyn + (size_t)st * TG::kStage, min(kBlk, len - j * kBlk),
-                                              sel_page[i], h, pooled_b0, C, lane);
-            fence_proxy_async_smem();  // these generic reads before the next TMA write of the stage
+        const uint32_t fill0 = fill;  // the first fill of this phase (the ring may hold descriptor chunks before)
+        auto refresh = [&](int i) {   // block at position i, all of whose fills have been issued
+            const int j = sel[i], valid = min(kBlk, len - j * kBlk);
+            RefreshAcc acc;
+            refresh_init(acc);
+            bool ok = true;
+#pragma unroll
+            for (int sb = 0; sb < kSub; ++sb) {
+                const uint32_t f = fill0 + (uint32_t)((i - i0) * kSub + sb);
+                if (lane == 0) ok = mbar_wait(&full[f % NSt], (f / NSt) & 1, c.status) && ok;
+                if (__shfl_sync(0xffffffffu, ok, 0))
+                    refresh_accum<kScorer>(acc, dyn + (size_t)(f % NSt) * TG::kStage, min(64, max(0, valid - 64 * sb)),
+                                           lane);
+            }
+            if (__shfl_sync(0xffffffffu, ok, 0))
+                refresh_finish<kScorer>(c, acc, valid, sel_page[i], h, pooled_b0, C, lane);
+            fence_proxy_async_smem();  // these generic reads before the next TMA writes of the stages
             __syncwarp();
         };
-        const uint32_t fill0 = fill;  // the first fill of this phase (the ring may hold descriptor chunks before)
-        for (int i = i0; i < i1; ++i, ++fill) {
-            const int st = fill % NSt;
-            if (fill >= (uint32_t)NSt) {
-                if (lane == 0 && alive) alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
-                alive = __shfl_sync(0xffffffffu, alive, 0);
-                if (alive && fill - NSt >= fill0 && touched(i - NSt)) {
-                    bool ok = true;  // (complete: the consumers released it)
-                    if (lane == 0) ok = mbar_wait(&full[st], ((fill / NSt) - 1) & 1, c.status);
-                    if (__shfl_sync(0xffffffffu, ok, 0)) refresh(i - NSt, st);
+        for (int i = i0; i < i1; ++i) {
+#pragma unroll 1
+            for (int sb = 0; sb < kSub; ++sb, ++fill) {
+                const int st = fill % NSt;
+                if (fill >= (uint32_t)NSt) {
+                    if (lane == 0 && alive) alive = mbar_wait(&empty[st], ((fill / NSt) - 1) & 1, c.status);
+                    alive = __shfl_sync(0xffffffffu, alive, 0);
+                    const uint32_t prev = fill - NSt;  // the fill whose stage is reused now
+                    if (alive && prev >= fill0 && (prev - fill0) % kSub == 0) {
+                        const int ip = i0 + (int)((prev - fill0) / kSub);
+                        if (touched(ip)) refresh(ip);
+                    }
                 }
-            }
-            if (lane == 0 && alive) {
-                {
+                if (lane == 0 && alive) {
                     const int j = sel[i];
                     const int pg = (j >= 0 && j < N) ? sel_page[i] : -1;
                     StageInfo inf;
                     inf.j = j;
-                    inf.valid = pg >= 0 ? min(kBlk, len - j * kBlk) : 0;
+                    inf.valid = pg >= 0 ? min(64, max(0, min(kBlk, len - j * kBlk) - 64 * sb)) : 0;
                     inf.ok = pg >= 0;
                     inf.pos = i;
                     info[st] = inf;
                     if (pg >= 0) {
                         uint8_t* base = dyn + (size_t)st * TG::kStage;
-                        const int y = (pg * c.H_kv + h) * kBlk;
+                        const int y = (pg * c.H_kv + h) * kBlk + 64 * sb;
                         mbar_arrive_expect_tx(&full[st], TG::kStage);
                         tma_load_2d(base, &tmK, &full[st], 0, y);
                         tma_load_2d(base + TG::kHalf, &tmK, &full[st], 64, y);
                         tma_load_2d(base + 2 * TG::kHalf, &tmV, &full[st], 0, y);
                         tma_load_2d(base + 3 * TG::kHalf, &tmV, &full[st], 64, y);
                     } else {
-                        report(c.status, SBA_DEV_BAD_SELECTION);
+                        if (sb == 0) report(c.status, SBA_DEV_BAD_SELECTION);
                         mbar_arrive(&full[st]);
                     }
                 }
+                __syncwarp();
             }
-            __syncwarp();
         }
-        for (int i = max(i0, i1 - NSt); i < i1; ++i) {
-            if (!alive || !touched(i)) continue;
-            const uint32_t f = fill0 + (uint32_t)(i - i0);
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(&full[f % NSt], (f / NSt) & 1, c.status);
-            if (__shfl_sync(0xffffffffu, ok, 0)) refresh(i, (int)(f % NSt));
+        // touched blocks whose first fill's stage was not reused in the loop
+        for (uint32_t prev = max(fill0, fill >= (uint32_t)NSt ? fill - NSt : 0u); prev < fill; ++prev) {
+            if (!alive || (prev - fill0) % kSub != 0) continue;
+            const int ip = i0 + (int)((prev - fill0) / kSub);
+            if (touched(ip)) refresh(ip);
         }
         named_sync(4, kThreads);  // the ring becomes the merge area
     } else {
@@ -1047,8 +1078,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         DecodeState dst;
         decode_state_init(dst);
         bool alive = true;
-        for (int i = i0; i < i1; ++i, ++fill) {
-            if ((int)(fill & 1) != grp) continue;  // the other group's block
+        for (int fi = 0; fi < (i1 - i0) * kSub; ++fi, ++fill) {
+            if ((int)(fill & 1) != grp) continue;  // the other group's fill
             const int st = fill % NSt;
             if (alive) alive = mbar_wait(&full[st], (fill / NSt) & 1, c.status);
             const StageInfo inf = info[st];
@@ -1061,12 +1092,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (rr < G) b0 = ld_peer_f32(peer_addr(u_s + rr * ustride + off, owner)) - lse_s[rr];
                     if (rr + 8 < G) b1 = ld_peer_f32(peer_addr(u_s + (rr + 8) * ustride + off, owner)) - lse_s[rr + 8];
                 }
-                if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && (lane & 3) == 0 && inf.pos < a.n_max) {
+                if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && (lane & 3) == 0 && inf.pos < a.n_max &&
+                    fi % kSub == 0) {
                     if (rr < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr) * a.n_max + inf.pos] = b0;
                     if (rr + 8 < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr + 8) * a.n_max + inf.pos] = b1;
                 }
                 if (alive)
-                    decode_block<kBlk>(dst, qa, stage, inf.valid, b0 * kLog2e, b1 * kLog2e, a.scale_log2, gw, lane);
+                    decode_block<64>(dst, qa, stage, inf.valid, b0 * kLog2e, b1 * kLog2e, a.scale_log2, gw, lane);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -1178,7 +1210,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     Plan pl{};
     pl.C = C;
     const int G = c.H_q / c.H_kv;
-    const int stage = c.b * kDescBytes;
+    const int stage = 64 * kDescBytes;  // a ring stage: 64 tokens of K and V, or 64 descriptors
     pl.slice = round4((c.max_blocks + C - 1) / C);
     pl.ccap = 1024;
     pl.sel_cap = round4(n_max_sel);
@@ -1190,7 +1222,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
         return o;
     };
     // the ring comes first (1024-aligned); the fallback selection reuses it
-    const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + (c.b == 64 ? 1 : 0);
+    const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + 1;
     int ns = 6;
     const int mb128 = (c.max_blocks + 127) & ~127;
     const int kall_words = p.scorer == SBA_SCORER_GATE ? 0 : mb128 + 4;  // (the gate's keys use the ring)
@@ -1293,8 +1325,9 @@ template <int kBlk, int kScorer, int kGM>
 int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaStream_t stream) {
     CUtensorMap tk, tv, td;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
-    if (!make_kv_tmap(&tk, c.k, rows, kBlk) || !make_kv_tmap(&tv, c.v, rows, kBlk)) return SBA_ERR_CUDA;
-    if (!make_desc_tmap(&td, kScorer == SBA_SCORER_QUEST ? c.desc : (void*)c.kg, (uint64_t)c.num_pages, c.H_kv, kBlk))
+    // boxes of 64 rows: 64 tokens of a (page, head) tile, or 64 descriptors
+    if (!make_kv_tmap(&tk, c.k, rows, 64) || !make_kv_tmap(&tv, c.v, rows, 64)) return SBA_ERR_CUDA;
+    if (!make_desc_tmap(&td, kScorer == SBA_SCORER_QUEST ? c.desc : (void*)c.kg, (uint64_t)c.num_pages, c.H_kv, 64))
         return SBA_ERR_CUDA;
     cudaError_t e = prepare_kernel<kBlk, kScorer, kGM>(pl.smem);
     if (e != cudaSuccess) {
