@@ -238,13 +238,14 @@ def build_layers(w, lay, seed, n_layers, dev):
     return layers, p, pos
 
 
-def layer_step(w, L, p, pos, q=None, k_new=None, v_new=None, path="fused"):
+def layer_step(w, L, p, pos, q=None, k_new=None, v_new=None, path="fused", out=None):
     from block_sparse_gqa_min_b200 import sba
 
     c, li, bufs = L["c"], L["li"], L["bufs"]
     q = li.q if q is None else q
     if path == "fused":
-        sba.sba_decode_step(c, q, p, w.scale, bufs.out, bufs.lse, k_new=li.k_new if k_new is None else k_new,
+        sba.sba_decode_step(c, q, p, w.scale, bufs.out if out is None else out, bufs.lse,
+                            k_new=li.k_new if k_new is None else k_new,
                             v_new=li.v_new if v_new is None else v_new, pos_start=pos, gate_A=L["A"],
                             sel_idx=bufs.sel_idx, sel_cnt=bufs.sel_cnt, gate_bias=bufs.gate_bias)
         return
@@ -389,27 +390,33 @@ def native(args, rank, world, local):
     # ---- e2e: host buffers, copies inside the timed region ----
     e2e = None
     if not args.no_e2e:
-        qh = [torch.empty_like(L["li"].q, device="cpu").pin_memory() for L in layers]
-        kh = [torch.empty_like(L["li"].k_new, device="cpu").pin_memory() for L in layers]
-        vh = [torch.empty_like(L["li"].v_new, device="cpu").pin_memory() for L in layers]
-        for i, L in enumerate(layers):
-            qh[i].copy_(L["li"].q)
-            kh[i].copy_(L["li"].k_new)
-            vh[i].copy_(L["li"].v_new)
-        oh = [torch.empty_like(L["bufs"].out, device="cpu").pin_memory() for L in layers]
-        qd = [torch.empty_like(L["li"].q) for L in layers]
-        kd = [torch.empty_like(L["li"].k_new) for L in layers]
-        vd = [torch.empty_like(L["li"].v_new) for L in layers]
-        h2d = sum(x.numel() * x.element_size() for x in qh + kh + vh)
-        d2h = sum(x.numel() * x.element_size() for x in oh)
+        # a step's inputs of every layer in one pinned host buffer per tensor, every layer's output
+        # back in one copy: one host-to-device copy per input tensor and one device-to-host copy
+        def stacked(ts):
+            h = torch.empty((len(ts),) + tuple(ts[0].shape), dtype=ts[0].dtype).pin_memory()
+            for i, t in enumerate(ts):
+                h[i].copy_(t)
+            return h, torch.empty(h.shape, dtype=h.dtype, device=dev)
+        qh, qd = stacked([L["li"].q for L in layers])
+        kh, kd = stacked([L["li"].k_new for L in layers])
+        vh, vd = stacked([L["li"].v_new for L in layers])
+        out0 = layers[0]["bufs"].out
+        od = torch.empty((len(layers),) + tuple(out0.shape), dtype=out0.dtype, device=dev)
+        oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
+        d2h = oh.numel() * oh.element_size()
 
         def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
             for i, L in enumerate(layers):
-                qd[i].copy_(qh[i], non_blocking=True)
-                kd[i].copy_(kh[i], non_blocking=True)
-                vd[i].copy_(vh[i], non_blocking=True)
-                layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i], path=args.path)
-                oh[i].copy_(L["bufs"].out, non_blocking=True)
+                if args.path == "fused":
+                    layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i], path="fused", out=od[i])
+                else:
+                    layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i], path=args.path)
+                    od[i].copy_(L["bufs"].out)
+            oh.copy_(od, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -426,7 +433,8 @@ def native(args, rank, world, local):
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
         e2e = {"value": round(job_gbs(step_bytes, world, t_e2e), 1), "unit": "GB/s",
                "ms_per_step": round(t_e2e, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "eager C-ABI calls per layer, pinned host q/k_new/v_new in, fp32 output out"}
+               "api": ("eager C-ABI call per layer; q, k_new, v_new of all layers from one pinned host buffer "
+                       "each (one copy per tensor per step), every layer's fp32 output back in one copy")}
 
     status = [int(L["c"].status.item()) for L in layers]
     if any(status):

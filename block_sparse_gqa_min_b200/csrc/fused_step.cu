@@ -29,6 +29,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <string.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "decode_tile.cuh"
@@ -1377,7 +1380,7 @@ int n_max_selected(const sba_cache& c, const sba_select_params& p) {
 
 }  // namespace
 
-int step_cluster_size(const sba_cache& c, const sba_select_params& p, int num_sms) {
+int step_cluster_size_uncached(const sba_cache& c, const sba_select_params& p, int num_sms) {
     // one CTA per SM: the largest C <= 16 with B*H_kv*C <= #SMs whose clusters are all
     // resident at once; failing that, the largest schedulable C
     const int64_t units = (int64_t)c.B * c.H_kv;
@@ -1391,6 +1394,52 @@ int step_cluster_size(const sba_cache& c, const sba_select_params& p, int num_sm
             if (active >= 1 && (pass == 1 || C == 1 || active >= units)) return C;
         }
     return 0;
+}
+
+// The choice above costs occupancy queries; it depends only on the device and the shapes, so
+// it is remembered (a small table, most recent first).
+int step_cluster_size(const sba_cache& c, const sba_select_params& p, int num_sms) {
+    struct Key {
+        int dev, sms, B, H_q, H_kv, b, max_blocks, max_len, n_budget, n_local, n_min, keep_num, keep_den, scorer;
+        bool operator==(const Key& o) const { return memcmp(this, &o, sizeof(Key)) == 0; }
+    };
+    static std::mutex mu;
+    static Key keys[16];
+    static int vals[16];
+    static int n = 0;
+    Key k;
+    memset(&k, 0, sizeof(k));
+    if (cudaGetDevice(&k.dev) != cudaSuccess) return 0;
+    k.sms = num_sms;
+    k.B = c.B;
+    k.H_q = c.H_q;
+    k.H_kv = c.H_kv;
+    k.b = c.b;
+    k.max_blocks = c.max_blocks;
+    k.max_len = c.max_len;
+    k.n_budget = p.n_budget;
+    k.n_local = p.n_local;
+    k.n_min = p.n_min;
+    k.keep_num = p.keep_num;
+    k.keep_den = p.keep_den;
+    k.scorer = p.scorer;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < n; ++i)
+            if (keys[i] == k) return vals[i];
+    }
+    const int C = step_cluster_size_uncached(c, p, num_sms);
+    if (C > 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        const int slot = n < 16 ? n++ : 15;
+        for (int i = slot; i > 0; --i) {
+            keys[i] = keys[i - 1];
+            vals[i] = vals[i - 1];
+        }
+        keys[0] = k;
+        vals[0] = C;
+    }
+    return C;
 }
 
 int launch_decode_step(const sba_cache& c, const void* q, const void* k_new, const void* v_new,

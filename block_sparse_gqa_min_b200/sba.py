@@ -180,9 +180,17 @@ class Cache:
         return int(self.seq_lens.shape[0])
 
     def struct(self) -> sba_cache:
-        return sba_cache(_ptr(self.k), _ptr(self.v), _ptr(self.block_table), _ptr(self.seq_lens),
-                         self.B, self.H_q, self.H_kv, self.d, self.b, self.max_blocks, self.num_pages,
-                         self.max_len, _ptr(self.desc), _ptr(self.kg), _ptr(self.status))
+        # rebuilt only when a tensor of the cache is replaced (in-place updates keep the pointers)
+        key = (id(self.k), id(self.v), id(self.block_table), id(self.seq_lens), id(self.desc), id(self.kg),
+               id(self.status), self.H_q, self.max_blocks, self.max_len)
+        cached = self.__dict__.get("_struct")
+        if cached is None or cached[0] != key:
+            st = sba_cache(_ptr(self.k), _ptr(self.v), _ptr(self.block_table), _ptr(self.seq_lens),
+                           self.B, self.H_q, self.H_kv, self.d, self.b, self.max_blocks, self.num_pages,
+                           self.max_len, _ptr(self.desc), _ptr(self.kg), _ptr(self.status))
+            cached = (key, st)
+            self.__dict__["_struct"] = cached
+        return cached[1]
 
 
 def select_params(n_budget=0, n_local=0, n_min=0, keep_num=0, keep_den=0, scorer=SBA_SCORER_QUEST):
