@@ -219,4 +219,182 @@ __device__ __forceinline__ void merge_warps(const float* merge_o, const float* m
     lse = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
 }
 
+
+// ---------------------------------------------------------------------------
+// Transposed tiles for at most 8*NH query heads (the fused step): the 16 tokens of a
+// warp are the MMA rows and the heads the columns -- S^T = K Q^T and O^T += V^T P^T --
+// so a group of G <= 8 heads fills one n8 tile instead of padding 16 rows, which halves
+// the tensor-core work and the O registers.  Blocks are staged 64 tokens at a time
+// (TileGeom<64>); P^T reaches the B-operand layout through movmatrix.
+// ---------------------------------------------------------------------------
+template <int NH>
+struct DecodeStateT {
+    float o[NH][8][4];  // O^T tile mt: c0,c1 = (channel 16mt + lane/4, heads 8nh + 2(lane%4) + 0/1); c2,c3 = channel + 8
+    float m[NH][2];     // running max (log2 units) of heads 8nh + 2(lane%4) + x
+    float l[NH][2];     // this lane's partial sums of those heads
+};
+
+template <int NH>
+__device__ __forceinline__ void decode_state_init_t(DecodeStateT<NH>& st) {
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) st.o[nh][mt][0] = st.o[nh][mt][1] = st.o[nh][mt][2] = st.o[nh][mt][3] = 0.f;
+        st.m[nh][0] = st.m[nh][1] = -INFINITY;
+        st.l[nh][0] = st.l[nh][1] = 0.f;
+    }
+}
+
+// Q of the group as B fragments of S^T = K Q^T: column = head 8nh + lane/4 (zero past G),
+// rows = channel pairs 16ks + 2(lane%4) (+8).
+template <int NH>
+__device__ __forceinline__ void load_q_frags_t(uint32_t (&qb)[NH][8][2], const __nv_bfloat16* qg, int G, int lane) {
+    const int c2 = (lane & 3) * 2;
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) {
+        const int head = nh * 8 + (lane >> 2);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const __nv_bfloat16* p = qg + head * kHeadDim + ks * 16 + c2;
+            qb[nh][ks][0] = head < G ? *reinterpret_cast<const uint32_t*>(p) : 0u;
+            qb[nh][ks][1] = head < G ? *reinterpret_cast<const uint32_t*>(p + 8) : 0u;
+        }
+    }
+}
+
+// One 64-token stage: the 16 tokens of token slot `slot` (0..3).  gb[nh][x] is the log-gate
+// (log2 units) of head 8nh + 2(lane%4) + x; `valid` counts the stage's valid tokens.
+template <int NH>
+__device__ __forceinline__ void decode_block_t(DecodeStateT<NH>& st, const uint32_t (&qb)[NH][8][2], uint8_t* stage,
+                                               int valid, const float (&gb)[NH][2], float scale_log2, int slot,
+                                               int lane) {
+    using TG = TileGeom<64>;
+    const int tok0 = slot * 16;
+    if (tok0 >= valid) return;
+    const uint32_t kb = smem_u32(stage);
+    const uint32_t vb = kb + 2 * TG::kHalf;
+    if (valid < tok0 + 16) {
+        // rows past len may hold anything: zero this warp's invalid V rows so 0*garbage cannot appear
+        uint8_t* vrow = stage + 2 * TG::kHalf;
+        for (int e = lane; e < (tok0 + 16 - valid) * 16; e += 32) {
+            const int row = valid + e / 16, ch = e % 16;
+            *reinterpret_cast<uint4*>(vrow + (ch >> 3) * TG::kHalf + row * 128 + ((ch & 7) << 4)) =
+                make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+    }
+    // ---- S^T = K Q^T (16 tokens x 8 heads per n-tile) ----
+    float s[NH][4];
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
+    {
+        const int row = tok0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const int chunk = 2 * ks + (lane >> 4);
+            uint32_t a[4];
+            ldmatrix_x4(swz(kb + (chunk >> 3) * TG::kHalf, row, chunk & 7), a[0], a[1], a[2], a[3]);
+#pragma unroll
+            for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(s[nh], a, qb[nh][ks][0], qb[nh][ks][1]);
+        }
+    }
+    // ---- scale, log-gate, mask; online softmax over the tokens of each head (base 2) ----
+    const int tr = lane >> 2;  // this lane's tokens: tr and tr + 8
+    const bool v0 = tok0 + tr < valid, v1 = tok0 + tr + 8 < valid;
+    bool rescale = false;
+    float alpha[NH][2], u[NH][2];
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            s[nh][x] = v0 ? fmaf(s[nh][x], scale_log2, gb[nh][x]) : -INFINITY;
+            s[nh][2 + x] = v1 ? fmaf(s[nh][2 + x], scale_log2, gb[nh][x]) : -INFINITY;
+            float mx = fmaxf(s[nh][x], s[nh][2 + x]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float n = fmaxf(st.m[nh][x], mx);
+            u[nh][x] = n == -INFINITY ? 0.f : n;
+            alpha[nh][x] = exp2f(st.m[nh][x] - u[nh][x]);
+            rescale |= alpha[nh][x] != 1.f;
+            st.m[nh][x] = n;
+            st.l[nh][x] *= alpha[nh][x];
+        }
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                st.o[nh][mt][0] *= alpha[nh][0];
+                st.o[nh][mt][1] *= alpha[nh][1];
+                st.o[nh][mt][2] *= alpha[nh][0];
+                st.o[nh][mt][3] *= alpha[nh][1];
+            }
+    }
+    // ---- P^T as B fragments (bf16 hi + lo): the two 8x8 halves of the S^T tile transposed ----
+    uint32_t bh[NH][2], bl[NH][2];
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) {
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[e] = exp2f(s[nh][e] - u[nh][e & 1]);
+        st.l[nh][0] += p[0] + p[2];
+        st.l[nh][1] += p[1] + p[3];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // tokens tr (hh = 0) and tr + 8 (hh = 1)
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(p[2 * hh], p[2 * hh + 1]);
+            const float2 hf = __bfloat1622float2(hi);
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(p[2 * hh] - hf.x, p[2 * hh + 1] - hf.y);
+            bh[nh][hh] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&hi));
+            bl[nh][hh] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&lo));
+        }
+    }
+    // ---- O^T += V^T P^T: eight 16-channel row tiles ----
+    {
+        const int q = lane >> 3;
+        const int row = tok0 + (q >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int chunk = 2 * mt + (q & 1);
+            uint32_t a[4];
+            ldmatrix_x4_trans(swz(vb + (chunk >> 3) * TG::kHalf, row, chunk & 7), a[0], a[1], a[2], a[3]);
+#pragma unroll
+            for (int nh = 0; nh < NH; ++nh) {
+                mma_bf16_16816(st.o[nh][mt], a, bh[nh][0], bh[nh][1]);
+                mma_bf16_16816(st.o[nh][mt], a, bl[nh][0], bl[nh][1]);
+            }
+        }
+    }
+}
+
+// This warp's (max, sum, O) of heads < G to shared memory in the layout of
+// decode_state_store: merge_o [warps][16][128], merge_ml [warps][16][2].
+template <int NH>
+__device__ __forceinline__ void decode_state_store_t(DecodeStateT<NH>& st, float* merge_o, float* merge_ml, int warp,
+                                                     int lane, int G) {
+    const int t = lane & 3, tr = lane >> 2;
+    float* mo = merge_o + warp * 16 * kHeadDim;
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            float l = st.l[nh][x];  // over the warp's tokens: lanes of equal lane%4 hold the same heads
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            const int hd = nh * 8 + 2 * t + x;
+            if (hd < G) {
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    mo[hd * kHeadDim + mt * 16 + tr] = st.o[nh][mt][x];
+                    mo[hd * kHeadDim + mt * 16 + tr + 8] = st.o[nh][mt][2 + x];
+                }
+                if (tr == 0) {
+                    merge_ml[(warp * 16 + hd) * 2] = st.m[nh][x];
+                    merge_ml[(warp * 16 + hd) * 2 + 1] = l;
+                }
+            }
+        }
+}
+
 }  // namespace sba

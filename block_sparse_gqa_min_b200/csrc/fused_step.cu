@@ -305,7 +305,7 @@ __device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
     return (p < 0 || p >= c.num_pages) ? -1 : (int)p;
 }
 
-template <int kBlk, int kScorer, int kGM>
+template <int kBlk, int kScorer, int kGM, int kNH>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmD, StepArgs a) {
@@ -1074,12 +1074,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_sync(4, kThreads);  // the ring becomes the merge area
     } else {
-        uint32_t qa[8][4];
-        load_q_frags(qa, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
-        const int rr = lane >> 2;
+        uint32_t qb[kNH][8][2];
+        load_q_frags_t<kNH>(qb, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
+        const int t4 = lane & 3;                      // this lane's heads: 8nh + 2*t4 + x
         const int grp = warp / kGW, gw = warp % kGW;  // consumer group, token slot
-        DecodeState dst;
-        decode_state_init(dst);
+        DecodeStateT<kNH> dst;
+        decode_state_init_t<kNH>(dst);
         bool alive = true;
         for (int fi = 0; fi < (i1 - i0) * kSub; ++fi, ++fill) {
             if ((int)(fill & 1) != grp) continue;  // the other group's fill
@@ -1088,27 +1088,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             const StageInfo inf = info[st];
             uint8_t* stage = dyn + (size_t)st * TG::kStage;
             if (inf.ok) {
-                // SAS log-gate of this block (natural log), 0 for the current block B0
-                float b0 = 0.f, b1 = 0.f;
+                // SAS log-gate of this block (natural log) for this lane's heads, 0 for the current
+                // block B0
+                float gb[kNH][2];
+#pragma unroll
+                for (int nh = 0; nh < kNH; ++nh) gb[nh][0] = gb[nh][1] = 0.f;
                 if (kScorer == SBA_SCORER_GATE && inf.j != N - 1) {
                     const int owner = inf.j / slice, off = inf.j - owner * slice;
-                    if (rr < G) b0 = ld_peer_f32(peer_addr(u_s + rr * ustride + off, owner)) - lse_s[rr];
-                    if (rr + 8 < G) b1 = ld_peer_f32(peer_addr(u_s + (rr + 8) * ustride + off, owner)) - lse_s[rr + 8];
+#pragma unroll
+                    for (int nh = 0; nh < kNH; ++nh)
+#pragma unroll
+                        for (int x = 0; x < 2; ++x) {
+                            const int hd = nh * 8 + 2 * t4 + x;
+                            if (hd < G) gb[nh][x] = ld_peer_f32(peer_addr(u_s + hd * ustride + off, owner)) - lse_s[hd];
+                        }
                 }
-                if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && (lane & 3) == 0 && inf.pos < a.n_max &&
+                if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && lane < 4 && inf.pos < a.n_max &&
                     fi % kSub == 0) {
-                    if (rr < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr) * a.n_max + inf.pos] = b0;
-                    if (rr + 8 < G) a.gate_bias[((int64_t)s * c.H_q + h * G + rr + 8) * a.n_max + inf.pos] = b1;
+#pragma unroll
+                    for (int nh = 0; nh < kNH; ++nh)
+#pragma unroll
+                        for (int x = 0; x < 2; ++x) {
+                            const int hd = nh * 8 + 2 * t4 + x;
+                            if (hd < G) a.gate_bias[((int64_t)s * c.H_q + h * G + hd) * a.n_max + inf.pos] = gb[nh][x];
+                        }
                 }
-                if (alive)
-                    decode_block<64>(dst, qa, stage, inf.valid, b0 * kLog2e, b1 * kLog2e, a.scale_log2, gw, lane);
+#pragma unroll
+                for (int nh = 0; nh < kNH; ++nh) gb[nh][0] *= kLog2e, gb[nh][1] *= kLog2e;
+                if (alive) decode_block_t<kNH>(dst, qb, stage, inf.valid, gb, a.scale_log2, gw, lane);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
         named_sync(4, kThreads);  // every consumer (and the producer) is done with the ring: it becomes the merge area
-        decode_state_store(dst, merge_o, merge_ml, warp, lane, G);
+        decode_state_store_t<kNH>(dst, merge_o, merge_ml, warp, lane, G);
         named_sync(3, kCW * 32);
         // per query row: the weight of each consumer warp's partial and the row's LSE over this
         // CTA's blocks (pushed to every CTA); kCW consecutive lanes per row
@@ -1255,10 +1269,10 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     return pl;
 }
 
-template <int kBlk, int kScorer, int kGM>
+template <int kBlk, int kScorer, int kGM, int kNH>
 cudaError_t prepare_kernel(int smem) {
-    auto kern = decode_step_kernel<kBlk, kScorer, kGM>;
-    if (allow_smem<decode_step_kernel<kBlk, kScorer, kGM>>(smem) != SBA_OK) return cudaErrorInvalidValue;
+    auto kern = decode_step_kernel<kBlk, kScorer, kGM, kNH>;
+    if (allow_smem<decode_step_kernel<kBlk, kScorer, kGM, kNH>>(smem) != SBA_OK) return cudaErrorInvalidValue;
     static bool nonportable_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1289,13 +1303,13 @@ cudaLaunchConfig_t step_config(const sba_cache& c, const Plan& pl, cudaStream_t 
 }
 
 // Clusters of this size the device can keep resident at once (0 if none).
-template <int kBlk, int kScorer, int kGM>
+template <int kBlk, int kScorer, int kGM, int kNH>
 int active_clusters(const sba_cache& c, const Plan& pl) {
-    if (prepare_kernel<kBlk, kScorer, kGM>(pl.smem) != cudaSuccess) return 0;
+    if (prepare_kernel<kBlk, kScorer, kGM, kNH>(pl.smem) != cudaSuccess) return 0;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = step_config(c, pl, nullptr, attr);
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, decode_step_kernel<kBlk, kScorer, kGM>, &cfg) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveClusters(&active, decode_step_kernel<kBlk, kScorer, kGM, kNH>, &cfg) != cudaSuccess) return 0;
     return active;
 }
 
@@ -1305,18 +1319,23 @@ template <class F>
 int dispatch(const sba_cache& c, const sba_select_params& p, F&& f) {
     const int G = c.H_q / c.H_kv;
     if (p.scorer == SBA_SCORER_QUEST)
-        return c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1>() : f.template run<128, SBA_SCORER_QUEST, 1>();
-    if (G <= 4) return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 4>() : f.template run<128, SBA_SCORER_GATE, 4>();
-    if (G <= 8) return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 8>() : f.template run<128, SBA_SCORER_GATE, 8>();
-    return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 16>() : f.template run<128, SBA_SCORER_GATE, 16>();
+        return G <= 8 ? (c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1, 1>()
+                                   : f.template run<128, SBA_SCORER_QUEST, 1, 1>())
+                      : (c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1, 2>()
+                                   : f.template run<128, SBA_SCORER_QUEST, 1, 2>());
+    if (G <= 4)
+        return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 4, 1>() : f.template run<128, SBA_SCORER_GATE, 4, 1>();
+    if (G <= 8)
+        return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 8, 1>() : f.template run<128, SBA_SCORER_GATE, 8, 1>();
+    return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 16, 2>() : f.template run<128, SBA_SCORER_GATE, 16, 2>();
 }
 
 struct ActiveClusters {
     const sba_cache& c;
     const Plan& pl;
-    template <int kBlk, int kScorer, int kGM>
+    template <int kBlk, int kScorer, int kGM, int kNH>
     int run() {
-        return active_clusters<kBlk, kScorer, kGM>(c, pl);
+        return active_clusters<kBlk, kScorer, kGM, kNH>(c, pl);
     }
 };
 
@@ -1324,7 +1343,7 @@ int active_clusters_any(const sba_cache& c, const sba_select_params& p, const Pl
     return dispatch(c, p, ActiveClusters{c, pl});
 }
 
-template <int kBlk, int kScorer, int kGM>
+template <int kBlk, int kScorer, int kGM, int kNH>
 int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaStream_t stream) {
     CUtensorMap tk, tv, td;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
@@ -1332,7 +1351,7 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     if (!make_kv_tmap(&tk, c.k, rows, 64) || !make_kv_tmap(&tv, c.v, rows, 64)) return SBA_ERR_CUDA;
     if (!make_desc_tmap(&td, kScorer == SBA_SCORER_QUEST ? c.desc : (void*)c.kg, (uint64_t)c.num_pages, c.H_kv, 64))
         return SBA_ERR_CUDA;
-    cudaError_t e = prepare_kernel<kBlk, kScorer, kGM>(pl.smem);
+    cudaError_t e = prepare_kernel<kBlk, kScorer, kGM, kNH>(pl.smem);
     if (e != cudaSuccess) {
         note_cuda_error(e);
         return SBA_ERR_CUDA;
@@ -1354,7 +1373,7 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     a.sel_cap = pl.sel_cap;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = step_config(c, pl, stream, attr);
-    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM>, tk, tv, td, a);
+    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM, kNH>, tk, tv, td, a);
     if (e != cudaSuccess) {
         note_cuda_error(e);
         return SBA_ERR_CUDA;
@@ -1367,9 +1386,9 @@ struct LaunchStep {
     const StepArgs& a;
     const Plan& pl;
     cudaStream_t stream;
-    template <int kBlk, int kScorer, int kGM>
+    template <int kBlk, int kScorer, int kGM, int kNH>
     int run() {
-        return launch_step_t<kBlk, kScorer, kGM>(c, a, pl, stream);
+        return launch_step_t<kBlk, kScorer, kGM, kNH>(c, a, pl, stream);
     }
 };
 
