@@ -367,13 +367,17 @@ __device__ __forceinline__ void decode_block_t(DecodeStateT<NH>& st, const uint3
     }
 }
 
-// This warp's (max, sum, O) of heads < G to shared memory in the layout of
-// decode_state_store: merge_o [warps][16][128], merge_ml [warps][16][2].
+// Row stride (floats) of merge_o for the transposed tiles: 4 words of padding put the eight
+// lanes of one head (consecutive channels) and the lanes of the next heads in distinct banks.
+constexpr int kMergeStride = kHeadDim + 4;
+
+// This warp's (max, sum, O) of heads < G to shared memory: merge_o [warps][16][kMergeStride]
+// (head rows, channels), merge_ml [warps][16][2].
 template <int NH>
 __device__ __forceinline__ void decode_state_store_t(DecodeStateT<NH>& st, float* merge_o, float* merge_ml, int warp,
                                                      int lane, int G) {
     const int t = lane & 3, tr = lane >> 2;
-    float* mo = merge_o + warp * 16 * kHeadDim;
+    float* mo = merge_o + warp * 16 * kMergeStride;
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
@@ -386,8 +390,8 @@ __device__ __forceinline__ void decode_state_store_t(DecodeStateT<NH>& st, float
             if (hd < G) {
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
-                    mo[hd * kHeadDim + mt * 16 + tr] = st.o[nh][mt][x];
-                    mo[hd * kHeadDim + mt * 16 + tr + 8] = st.o[nh][mt][2 + x];
+                    mo[hd * kMergeStride + mt * 16 + tr] = st.o[nh][mt][x];
+                    mo[hd * kMergeStride + mt * 16 + tr + 8] = st.o[nh][mt][2 + x];
                 }
                 if (tr == 0) {
                     merge_ml[(warp * 16 + hd) * 2] = st.m[nh][x];

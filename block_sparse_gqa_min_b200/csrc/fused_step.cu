@@ -320,8 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ uint32_t sh[2];
     __shared__ int misc[4];
     __shared__ float lse_s[kMaxGroup];
-    __shared__ __align__(16) float wgt_s[kMaxGroup][kCW];  // merge weights of the consumer warps
     __shared__ float lse_all[kMaxCluster * kMaxGroup];
+    __shared__ __align__(16) float wgt_s[kMaxGroup][kCW];  // merge weights of the consumer warps
+    __shared__ float cw_s[kMaxGroup][kMaxCluster];       // merge weights of the cluster's CTAs
+    __shared__ float rlse_s[kMaxGroup];
     __shared__ float mz_all[kMaxCluster * kMaxGroup][2];
     __shared__ int local_page[kMaxLocal];
     __shared__ __align__(16) float pooled[3 * kHeadDim];     // refresh-before-score scratch
@@ -342,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     StageInfo* info = reinterpret_cast<StageInfo*>(empty + NSt);
     // after the decode: per-warp merge area (aliases the ring)
     float* merge_o = reinterpret_cast<float*>(dyn);
-    float* merge_ml = merge_o + kCW * 16 * kHeadDim;
+    float* merge_ml = merge_o + kCW * 16 * kMergeStride;
 
     const sba_cache& c = a.c;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1150,15 +1152,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row = e / kHeadDim, ch = e % kHeadDim;
             const float4 w0 = *reinterpret_cast<const float4*>(&wgt_s[row][0]);
             const float4 w1 = *reinterpret_cast<const float4*>(&wgt_s[row][4]);
-            const float* mo = merge_o + row * kHeadDim + ch;
+            const float* mo = merge_o + row * kMergeStride + ch;
             float o = w0.x * mo[0];
-            o = fmaf(w0.y, mo[1 * 16 * kHeadDim], o);
-            o = fmaf(w0.z, mo[2 * 16 * kHeadDim], o);
-            o = fmaf(w0.w, mo[3 * 16 * kHeadDim], o);
-            o = fmaf(w1.x, mo[4 * 16 * kHeadDim], o);
-            o = fmaf(w1.y, mo[5 * 16 * kHeadDim], o);
-            o = fmaf(w1.z, mo[6 * 16 * kHeadDim], o);
-            o = fmaf(w1.w, mo[7 * 16 * kHeadDim], o);
+            o = fmaf(w0.y, mo[1 * 16 * kMergeStride], o);
+            o = fmaf(w0.z, mo[2 * 16 * kMergeStride], o);
+            o = fmaf(w0.w, mo[3 * 16 * kMergeStride], o);
+            o = fmaf(w1.x, mo[4 * 16 * kMergeStride], o);
+            o = fmaf(w1.y, mo[5 * 16 * kMergeStride], o);
+            o = fmaf(w1.z, mo[6 * 16 * kMergeStride], o);
+            o = fmaf(w1.w, mo[7 * 16 * kMergeStride], o);
             const int p = e / share;
             st_peer_f32(peer_addr(recv_o + r * share + (e - p * share), p), o);
         }
@@ -1167,28 +1169,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- phase 4: merge the cluster's partials (local data only) ----------------
     cluster_sync();  // every partial pushed; no shared memory is read remotely after this
     {
+        // the weight of every CTA's partial in each row of my share (16 lanes per row, lane p for
+        // CTA p), then every element of the share as the weighted sum of the C partials
         const int e0 = r * share, e1 = min(e0 + share, E);
-        for (int e = e0 + tid; e < e1; e += kThreads) {
-            const int row = e / kHeadDim, ch = e % kHeadDim;
-            float M = -INFINITY;
-            for (int p = 0; p < C; ++p) M = fmaxf(M, lse_all[p * G + row]);
-            float o = 0.f, W = 0.f;
-            if (M > -INFINITY) {
-                for (int p = 0; p < C; ++p) {
-                    const float l = lse_all[p * G + row];
-                    if (l == -INFINITY) continue;
-                    const float wgt = expf(l - M);
-                    W += wgt;
-                    o = fmaf(wgt, recv_o[p * share + (e - e0)], o);
-                }
-                o /= W;
+        const int rw0 = e0 / kHeadDim, nrw = e1 > e0 ? (e1 - 1) / kHeadDim - rw0 + 1 : 0;
+        for (int rp = warp; 2 * rp < nrw; rp += kThreads / 32) {  // (warp-uniform: whole warps shuffle)
+            const int rl = 2 * rp + (lane >> 4), p = lane & 15;
+            const float l = (rl < nrw && p < C) ? lse_all[p * G + rw0 + rl] : -INFINITY;
+            float M = l;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            const float w = M > -INFINITY ? expf(l - M) : 0.f;
+            float W = w;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+            if (rl < nrw) {
+                cw_s[rl][p] = W > 0.f ? w / W : 0.f;
+                if (p == 0) rlse_s[rl] = W > 0.f ? M + logf(W) : -INFINITY;
             }
+        }
+        __syncthreads();
+        for (int e = e0 + tid; e < e1; e += kThreads) {
+            const int row = e / kHeadDim, ch = e % kHeadDim, rl = row - rw0;
+            float o = 0.f;
+#pragma unroll
+            for (int p = 0; p < kMaxCluster; ++p)
+                if (p < C) o = fmaf(cw_s[rl][p], recv_o[p * share + (e - e0)], o);
             const int64_t orow = (int64_t)s * c.H_q + h * G + row;
             if (a.out_dtype == SBA_OUT_BF16)
                 reinterpret_cast<__nv_bfloat16*>(a.out)[orow * kHeadDim + ch] = __float2bfloat16_rn(o);
             else
                 reinterpret_cast<float*>(a.out)[orow * kHeadDim + ch] = o;
-            if (ch == 0 && a.lse_out) a.lse_out[orow] = W > 0.f ? M + logf(W) : -INFINITY;
+            if (ch == 0 && a.lse_out) a.lse_out[orow] = rlse_s[rl];
         }
     }
     if (kScorer == SBA_SCORER_GATE && tile_refresh && N >= 1 && tb1 == N - 1) {
@@ -1239,7 +1251,7 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
         return o;
     };
     // the ring comes first (1024-aligned); the fallback selection reuses it
-    const int min_stages = (kCW * 16 * kHeadDim * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + 1;
+    const int min_stages = (kCW * 16 * kMergeStride * 4 + kCW * 16 * 2 * 4 + stage - 1) / stage + 1;
     int ns = 6;
     const int mb128 = (c.max_blocks + 127) & ~127;
     const int kall_words = p.scorer == SBA_SCORER_GATE ? 0 : mb128 + 4;  // (the gate's keys use the ring)
