@@ -136,7 +136,7 @@ __device__ __forceinline__ void append_store(const StepArgs& a, int s, int h, in
 }
 
 // Elements [e0, e1) of the step's new rows, written through the block table.
-__device__ void append_rows(const StepArgs& a, int s, int h, int p0, int e0, int e1, int tid) {
+__device__ __noinline__ void append_rows(const StepArgs& a, int s, int h, int p0, int e0, int e1, int tid) {
     for (int e = e0 + tid; e < e1; e += kThreads) append_store(a, s, h, p0, e, __ldg(append_src(a, s, h, e)));
     fence_proxy_async_global();
 }
@@ -144,7 +144,7 @@ __device__ void append_rows(const StepArgs& a, int s, int h, int p0, int e0, int
 // Descriptor of block j of (s, h) from global memory (threads 0..127, one
 // channel each).  Quest: min/max rows; gate: pooled -> kg = A pooled.
 template <int kScorer>
-__device__ void refresh_from_global(const StepArgs& a, int s, int h, int j, int len, float* pooled, int tid) {
+__device__ __noinline__ void refresh_from_global(const StepArgs& a, int s, int h, int j, int len, float* pooled, int tid) {
     const sba_cache& c = a.c;
     const int64_t page = page_of(c, s, j, tid == 0 ? c.status : nullptr);
     const int cnt = min(c.b, len - j * c.b);
@@ -308,7 +308,7 @@ __device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
 template <int kBlk, int kScorer, int kGM, int kNH>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                       const __grid_constant__ CUtensorMap tmD, StepArgs a) {
+                       const __grid_constant__ CUtensorMap tmD, const __grid_constant__ StepArgs a) {
     // The ring holds 64-token stages (32 KB): a block of 128 tokens takes two consecutive fills,
     // and a descriptor chunk is 64 descriptors.
     using TG = TileGeom<64>;

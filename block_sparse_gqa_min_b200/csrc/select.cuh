@@ -162,7 +162,7 @@ __device__ void select_and_compact(const uint32_t* keys, int NC, int N, int k, i
 // words, bkey/bidx/brank [cap] words each, misc [2] ints.
 // ---------------------------------------------------------------------------
 template <int kNT>
-__device__ void select_fast(const uint32_t* keys, int NC, int N, int k, int32_t* out, int n_max, uint32_t* gmax,
+__device__ __noinline__ void select_fast(const uint32_t* keys, int NC, int N, int k, int32_t* out, int n_max, uint32_t* gmax,
                             uint32_t* bkey, int* bidx, int* brank, int cap, int* misc, uint32_t* hist, int* warp_tot,
                             uint32_t* sh) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
