@@ -305,6 +305,112 @@ __device__ __forceinline__ int page_quiet(const sba_cache& c, int s, int j) {
     return (p < 0 || p >= c.num_pages) ? -1 : (int)p;
 }
 
+// Paged cache scoring of blocks [j0, js1) (their pages in `pages`): Quest keys into `keys` and
+// every CTA's `kall`, or the gate's u into u_s.  Out of line: a contiguous cache never runs it.
+template <int kScorer, int kGM>
+__device__ __noinline__ void score_paged(const StepArgs& a, int s, int h, int G, int j0, int js1, const int* pages,
+                                         uint32_t* keys, uint32_t* kall, bool trivial, int C, float* u_s, int ustride,
+                                         int warp, int lane) {
+    const sba_cache& c = a.c;
+    // Paged cache: every warp streams descriptors straight into registers: kRB blocks per
+    // warp and round, lane l holding bytes [16 l, 16 l + 16) of each 512-byte descriptor;
+    // the next round's loads are in flight while the current round is reduced.
+
+        constexpr int kNW = kThreads / 32;
+        constexpr int kRB = (kScorer == SBA_SCORER_GATE && kGM > 8) ? 4 : 8;  // (register budget)
+        const uint8_t* src = (kScorer == SBA_SCORER_QUEST ? reinterpret_cast<const uint8_t*>(c.desc)
+                                                          : reinterpret_cast<const uint8_t*>(c.kg)) +
+                             (int64_t)h * kDescBytes + lane * 16;
+        const int64_t pstride = (int64_t)c.H_kv * kDescBytes;
+        float coef[8];
+        float qg[kGM][4];  // gate: kGM = G rounded up to a power of two
+        if (kScorer == SBA_SCORER_QUEST) {
+            quest_coef(coef, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
+        } else {
+            // gate: lane owns channels 4*lane..4*lane+3 of the fp32 gate key
+#pragma unroll
+            for (int g = 0; g < kGM; ++g) {
+                if (g < G) {
+                    const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim +
+                                                                        4 * lane));
+                    qg[g][0] = bf16_lo(w.x);
+                    qg[g][1] = bf16_hi(w.x);
+                    qg[g][2] = bf16_lo(w.y);
+                    qg[g][3] = bf16_hi(w.y);
+                } else {
+                    qg[g][0] = qg[g][1] = qg[g][2] = qg[g][3] = 0.f;
+                }
+            }
+        }
+        uint4 wc[kRB], wn[kRB];
+        auto load_round = [&](int base, uint4(&w)[kRB]) {
+#pragma unroll
+            for (int b = 0; b < kRB; ++b) {
+                const int j = base + b;
+                const int pg = j < js1 ? pages[j - j0] : -1;
+                w[b] = pg >= 0 ? ld_stream_v4(src + pg * pstride) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        int base = j0 + warp * kRB;
+        if (base < js1) load_round(base, wc);
+        for (; base < js1; base += kNW * kRB) {
+            if (base + kNW * kRB < js1) load_round(base + kNW * kRB, wn);
+            if (kScorer == SBA_SCORER_QUEST) {
+                float part[kRB][1];
+#pragma unroll
+                for (int b = 0; b < kRB; ++b) {
+                    const uint32_t ws[4] = {wc[b].x, wc[b].y, wc[b].z, wc[b].w};
+                    float acc = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc = fmaf(coef[2 * e], bf16_lo(ws[e]), acc);
+                        acc = fmaf(coef[2 * e + 1], bf16_hi(ws[e]), acc);
+                    }
+                    part[b][0] = acc;
+                }
+                float tot[1];
+                reduce_scatter<kRB, 1>(part, tot, lane);
+                const int j = base + rs_block<kRB>(lane);
+                if ((lane & 3) == 0 && j < js1) {
+                    const uint32_t key = pages[j - j0] >= 0 ? orderable_key(tot[0]) : 0u;
+                    keys[j - j0] = key;
+                    if (!trivial)
+                        for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(kall + j, p), key);
+                }
+            } else {
+#pragma unroll
+                for (int q4 = 0; q4 < kRB; q4 += 4) {
+                    float part[4][kGM];
+#pragma unroll
+                    for (int b4 = 0; b4 < 4; ++b4) {
+                        const uint4 w = wc[q4 + b4];
+                        const float x0 = __uint_as_float(w.x), x1 = __uint_as_float(w.y), x2 = __uint_as_float(w.z),
+                                    x3 = __uint_as_float(w.w);
+#pragma unroll
+                        for (int g = 0; g < kGM; ++g) {
+                            float acc = qg[g][0] * x0;
+                            acc = fmaf(qg[g][1], x1, acc);
+                            acc = fmaf(qg[g][2], x2, acc);
+                            acc = fmaf(qg[g][3], x3, acc);
+                            part[b4][g] = acc;
+                        }
+                    }
+                    float tot[kGM];
+                    reduce_scatter<4, kGM>(part, tot, lane);
+                    const int j = base + q4 + rs_block<4>(lane);
+                    if ((lane & 7) == 0 && j < js1) {
+                        const bool ok = pages[j - j0] >= 0;
+#pragma unroll
+                        for (int g = 0; g < kGM; ++g)
+                            if (g < G) u_s[g * ustride + (j - j0)] = ok ? tot[g] : -INFINITY;
+                    }
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < kRB; ++b) wc[b] = wn[b];
+        }
+}
+
 template <int kBlk, int kScorer, int kGM, int kNH>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -641,103 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fill = (uint32_t)ntot;
     } else {
-    // Paged cache: every warp streams descriptors straight into registers: kRB blocks per
-    // warp and round, lane l holding bytes [16 l, 16 l + 16) of each 512-byte descriptor;
-    // the next round's loads are in flight while the current round is reduced.
-
-        constexpr int kNW = kThreads / 32;
-        constexpr int kRB = (kScorer == SBA_SCORER_GATE && kGM > 8) ? 4 : 8;  // (register budget)
-        const uint8_t* src = (kScorer == SBA_SCORER_QUEST ? reinterpret_cast<const uint8_t*>(c.desc)
-                                                          : reinterpret_cast<const uint8_t*>(c.kg)) +
-                             (int64_t)h * kDescBytes + lane * 16;
-        const int64_t pstride = (int64_t)c.H_kv * kDescBytes;
-        float coef[8];
-        float qg[kGM][4];  // gate: kGM = G rounded up to a power of two
-        if (kScorer == SBA_SCORER_QUEST) {
-            quest_coef(coef, a.q + ((int64_t)s * c.H_q + h * G) * kHeadDim, G, lane);
-        } else {
-            // gate: lane owns channels 4*lane..4*lane+3 of the fp32 gate key
-#pragma unroll
-            for (int g = 0; g < kGM; ++g) {
-                if (g < G) {
-                    const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim +
-                                                                        4 * lane));
-                    qg[g][0] = bf16_lo(w.x);
-                    qg[g][1] = bf16_hi(w.x);
-                    qg[g][2] = bf16_lo(w.y);
-                    qg[g][3] = bf16_hi(w.y);
-                } else {
-                    qg[g][0] = qg[g][1] = qg[g][2] = qg[g][3] = 0.f;
-                }
-            }
-        }
-        uint4 wc[kRB], wn[kRB];
-        auto load_round = [&](int base, uint4(&w)[kRB]) {
-#pragma unroll
-            for (int b = 0; b < kRB; ++b) {
-                const int j = base + b;
-                const int pg = j < js1 ? pages[j - j0] : -1;
-                w[b] = pg >= 0 ? ld_stream_v4(src + pg * pstride) : make_uint4(0u, 0u, 0u, 0u);
-            }
-        };
-        int base = j0 + warp * kRB;
-        if (base < js1) load_round(base, wc);
-        for (; base < js1; base += kNW * kRB) {
-            if (base + kNW * kRB < js1) load_round(base + kNW * kRB, wn);
-            if (kScorer == SBA_SCORER_QUEST) {
-                float part[kRB][1];
-#pragma unroll
-                for (int b = 0; b < kRB; ++b) {
-                    const uint32_t ws[4] = {wc[b].x, wc[b].y, wc[b].z, wc[b].w};
-                    float acc = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        acc = fmaf(coef[2 * e], bf16_lo(ws[e]), acc);
-                        acc = fmaf(coef[2 * e + 1], bf16_hi(ws[e]), acc);
-                    }
-                    part[b][0] = acc;
-                }
-                float tot[1];
-                reduce_scatter<kRB, 1>(part, tot, lane);
-                const int j = base + rs_block<kRB>(lane);
-                if ((lane & 3) == 0 && j < js1) {
-                    const uint32_t key = pages[j - j0] >= 0 ? orderable_key(tot[0]) : 0u;
-                    keys[j - j0] = key;
-                    if (!trivial)
-                        for (int p = 0; p < C; ++p) st_peer_u32(peer_addr(kall + j, p), key);
-                }
-            } else {
-#pragma unroll
-                for (int q4 = 0; q4 < kRB; q4 += 4) {
-                    float part[4][kGM];
-#pragma unroll
-                    for (int b4 = 0; b4 < 4; ++b4) {
-                        const uint4 w = wc[q4 + b4];
-                        const float x0 = __uint_as_float(w.x), x1 = __uint_as_float(w.y), x2 = __uint_as_float(w.z),
-                                    x3 = __uint_as_float(w.w);
-#pragma unroll
-                        for (int g = 0; g < kGM; ++g) {
-                            float acc = qg[g][0] * x0;
-                            acc = fmaf(qg[g][1], x1, acc);
-                            acc = fmaf(qg[g][2], x2, acc);
-                            acc = fmaf(qg[g][3], x3, acc);
-                            part[b4][g] = acc;
-                        }
-                    }
-                    float tot[kGM];
-                    reduce_scatter<4, kGM>(part, tot, lane);
-                    const int j = base + q4 + rs_block<4>(lane);
-                    if ((lane & 7) == 0 && j < js1) {
-                        const bool ok = pages[j - j0] >= 0;
-#pragma unroll
-                        for (int g = 0; g < kGM; ++g)
-                            if (g < G) u_s[g * ustride + (j - j0)] = ok ? tot[g] : -INFINITY;
-                    }
-                }
-            }
-#pragma unroll
-            for (int b = 0; b < kRB; ++b) wc[b] = wn[b];
-        }
+        score_paged<kScorer, kGM>(a, s, h, G, j0, js1, pages, keys, kall, trivial, C, u_s, ustride, warp, lane);
     }
     __syncthreads();
     if (app_e >= 0) append_store(a, s, h, p0, app_e, app_v);  // (its proxy fence comes before barrier B)
