@@ -411,7 +411,7 @@ __device__ __noinline__ void score_paged(const StepArgs& a, int s, int h, int G,
         }
 }
 
-template <int kBlk, int kScorer, int kGM, int kNH>
+template <int kBlk, int kScorer, int kGM, int kNH, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmD, const __grid_constant__ StepArgs a) {
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kProducer && lane == 0) {
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
-        if (c.block_table == nullptr) prefetch_tmap(&tmD);
+        if (!kPaged) prefetch_tmap(&tmD);
     }
     __syncthreads();
     pdl_wait();
@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int p0raw = a.n_new > 0 ? __ldg(a.pos_start + s) : 0;
     // A contiguous cache's descriptors need no length to be located: the first ring stages of
     // this CTA's slice (a fixed share of max_blocks) are requested before the lengths arrive.
-    const bool contiguous = c.block_table == nullptr;
+    constexpr bool contiguous = !kPaged;
     const int nspec = contiguous ? min(NSt, (a.slice + kSC - 1) / kSC) : 0;
     if (contiguous && warp == kProducer && lane == 0)
         for (int f = 0; f < nspec; ++f) {
@@ -599,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- phase 1: score this CTA's slice ----------------
     __syncthreads();  // page ids of the slice
     uint32_t fill = 0;  // ring fills so far (consecutive fills alternate consumer groups)
-    if (c.block_table == nullptr) {
+    if (!kPaged) {
         // Contiguous cache: one TMA load brings the descriptors of kBlk consecutive blocks into
         // a ring stage (128-byte quarter rows, 128-byte swizzle); the two consumer groups take
         // alternate stages, each warp 16 descriptors (one tensor-core tile for the gate) per
@@ -980,7 +980,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = tid; i < k; i += kThreads) {
             const int j = sel[i];
             const int p = j / slice;
-            sel_page[i] = c.block_table == nullptr ? page_quiet(c, s, j)
+            sel_page[i] = !kPaged ? page_quiet(c, s, j)
                           : p == r                 ? pages[j - j0]
                                                    : (int)ld_peer_u32(peer_addr(pages + (j - p * slice), p));
         }
@@ -1291,10 +1291,10 @@ Plan plan_step(const sba_cache& c, const sba_select_params& p, int C, int n_max_
     return pl;
 }
 
-template <int kBlk, int kScorer, int kGM, int kNH>
+template <int kBlk, int kScorer, int kGM, int kNH, bool kPaged>
 cudaError_t prepare_kernel(int smem) {
-    auto kern = decode_step_kernel<kBlk, kScorer, kGM, kNH>;
-    if (allow_smem<decode_step_kernel<kBlk, kScorer, kGM, kNH>>(smem) != SBA_OK) return cudaErrorInvalidValue;
+    auto kern = decode_step_kernel<kBlk, kScorer, kGM, kNH, kPaged>;
+    if (allow_smem<decode_step_kernel<kBlk, kScorer, kGM, kNH, kPaged>>(smem) != SBA_OK) return cudaErrorInvalidValue;
     static bool nonportable_set[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1325,39 +1325,48 @@ cudaLaunchConfig_t step_config(const sba_cache& c, const Plan& pl, cudaStream_t 
 }
 
 // Clusters of this size the device can keep resident at once (0 if none).
-template <int kBlk, int kScorer, int kGM, int kNH>
+template <int kBlk, int kScorer, int kGM, int kNH, bool kPaged>
 int active_clusters(const sba_cache& c, const Plan& pl) {
-    if (prepare_kernel<kBlk, kScorer, kGM, kNH>(pl.smem) != cudaSuccess) return 0;
+    if (prepare_kernel<kBlk, kScorer, kGM, kNH, kPaged>(pl.smem) != cudaSuccess) return 0;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = step_config(c, pl, nullptr, attr);
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, decode_step_kernel<kBlk, kScorer, kGM, kNH>, &cfg) != cudaSuccess) return 0;
+    if (cudaOccupancyMaxActiveClusters(&active, decode_step_kernel<kBlk, kScorer, kGM, kNH, kPaged>, &cfg) != cudaSuccess) return 0;
     return active;
 }
 
-// Kernel instantiation for a cache shape: block size, scorer, and (gate) the
-// head count rounded up to a power of two.
-template <class F>
-int dispatch(const sba_cache& c, const sba_select_params& p, F&& f) {
+template <bool kPaged, class F>
+int dispatch_shape(const sba_cache& c, const sba_select_params& p, F&& f) {
     const int G = c.H_q / c.H_kv;
     if (p.scorer == SBA_SCORER_QUEST)
-        return G <= 8 ? (c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1, 1>()
-                                   : f.template run<128, SBA_SCORER_QUEST, 1, 1>())
-                      : (c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1, 2>()
-                                   : f.template run<128, SBA_SCORER_QUEST, 1, 2>());
+        return G <= 8 ? (c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1, 1, kPaged>()
+                                   : f.template run<128, SBA_SCORER_QUEST, 1, 1, kPaged>())
+                      : (c.b == 64 ? f.template run<64, SBA_SCORER_QUEST, 1, 2, kPaged>()
+                                   : f.template run<128, SBA_SCORER_QUEST, 1, 2, kPaged>());
     if (G <= 4)
-        return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 4, 1>() : f.template run<128, SBA_SCORER_GATE, 4, 1>();
+        return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 4, 1, kPaged>()
+                         : f.template run<128, SBA_SCORER_GATE, 4, 1, kPaged>();
     if (G <= 8)
-        return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 8, 1>() : f.template run<128, SBA_SCORER_GATE, 8, 1>();
-    return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 16, 2>() : f.template run<128, SBA_SCORER_GATE, 16, 2>();
+        return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 8, 1, kPaged>()
+                         : f.template run<128, SBA_SCORER_GATE, 8, 1, kPaged>();
+    return c.b == 64 ? f.template run<64, SBA_SCORER_GATE, 16, 2, kPaged>()
+                     : f.template run<128, SBA_SCORER_GATE, 16, 2, kPaged>();
+}
+
+// Kernel instantiation for a cache shape: block size, scorer, (gate) the head count rounded
+// up to a power of two, and whether pages go through a block table (each variant holds only
+// the scoring path it runs).
+template <class F>
+int dispatch(const sba_cache& c, const sba_select_params& p, F&& f) {
+    return c.block_table != nullptr ? dispatch_shape<true>(c, p, f) : dispatch_shape<false>(c, p, f);
 }
 
 struct ActiveClusters {
     const sba_cache& c;
     const Plan& pl;
-    template <int kBlk, int kScorer, int kGM, int kNH>
+    template <int kBlk, int kScorer, int kGM, int kNH, bool kPaged>
     int run() {
-        return active_clusters<kBlk, kScorer, kGM, kNH>(c, pl);
+        return active_clusters<kBlk, kScorer, kGM, kNH, kPaged>(c, pl);
     }
 };
 
@@ -1365,7 +1374,7 @@ int active_clusters_any(const sba_cache& c, const sba_select_params& p, const Pl
     return dispatch(c, p, ActiveClusters{c, pl});
 }
 
-template <int kBlk, int kScorer, int kGM, int kNH>
+template <int kBlk, int kScorer, int kGM, int kNH, bool kPaged>
 int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaStream_t stream) {
     CUtensorMap tk, tv, td;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
@@ -1373,7 +1382,7 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     if (!make_kv_tmap(&tk, c.k, rows, 64) || !make_kv_tmap(&tv, c.v, rows, 64)) return SBA_ERR_CUDA;
     if (!make_desc_tmap(&td, kScorer == SBA_SCORER_QUEST ? c.desc : (void*)c.kg, (uint64_t)c.num_pages, c.H_kv, 64))
         return SBA_ERR_CUDA;
-    cudaError_t e = prepare_kernel<kBlk, kScorer, kGM, kNH>(pl.smem);
+    cudaError_t e = prepare_kernel<kBlk, kScorer, kGM, kNH, kPaged>(pl.smem);
     if (e != cudaSuccess) {
         note_cuda_error(e);
         return SBA_ERR_CUDA;
@@ -1395,7 +1404,7 @@ int launch_step_t(const sba_cache& c, const StepArgs& a0, const Plan& pl, cudaSt
     a.sel_cap = pl.sel_cap;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = step_config(c, pl, stream, attr);
-    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM, kNH>, tk, tv, td, a);
+    e = cudaLaunchKernelEx(&cfg, decode_step_kernel<kBlk, kScorer, kGM, kNH, kPaged>, tk, tv, td, a);
     if (e != cudaSuccess) {
         note_cuda_error(e);
         return SBA_ERR_CUDA;
@@ -1408,9 +1417,9 @@ struct LaunchStep {
     const StepArgs& a;
     const Plan& pl;
     cudaStream_t stream;
-    template <int kBlk, int kScorer, int kGM, int kNH>
+    template <int kBlk, int kScorer, int kGM, int kNH, bool kPaged>
     int run() {
-        return launch_step_t<kBlk, kScorer, kGM, kNH>(c, a, pl, stream);
+        return launch_step_t<kBlk, kScorer, kGM, kNH, kPaged>(c, a, pl, stream);
     }
 };
 
