@@ -17,7 +17,8 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 
-def run_fused(w: W.Workload, seed=0, n_app=0, layout=None, layer_inputs=None, device="cpu", out_dtype=torch.float32):
+def run_fused(w: W.Workload, seed=0, n_app=0, layout=None, layer_inputs=None, device="cpu", out_dtype=torch.float32,
+              pos_back=0):
     lay = layout or W.make_layout(w, seed, device=device)
     li = layer_inputs or W.make_layer(w, lay, seed, 0, device=device)
     c = gpu_cache(w, lay, li)
@@ -40,7 +41,7 @@ def run_fused(w: W.Workload, seed=0, n_app=0, layout=None, layer_inputs=None, de
         g = torch.Generator().manual_seed(seed + 77)
         kw = dict(k_new=torch.randn((w.B, n_app, w.H_kv, w.d), generator=g).to(torch.bfloat16).to(dev),
                   v_new=torch.randn((w.B, n_app, w.H_kv, w.d), generator=g).to(torch.bfloat16).to(dev),
-                  pos_start=(c.seq_lens - n_app).clamp(min=0).to(torch.int32))
+                  pos_start=(c.seq_lens - n_app - pos_back).clamp(min=0).to(torch.int32))
     sba.sba_decode_step(c, li.q.to(dev), p, w.scale, out, lse, gate_A=A, sel_idx=sel_idx, sel_cnt=sel_cnt,
                         gate_bias=gbias, **kw)
     torch.cuda.synchronize()
@@ -112,6 +113,14 @@ def test_fused_refreshes_scored_block_first():
     w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=3000, len_hi=3000, n_budget=6, n_local=0)
     run_fused(w, seed=2, n_app=1)
     run_fused(w, seed=3, n_app=40)
+
+
+def test_fused_refresh_inside_fill_loop():
+    """Tokens overwritten inside an early local block (12 local blocks, two CTAs per
+    cluster): the touched block is followed by more fills than the ring holds, so its
+    descriptor is rebuilt inside the producer's fill loop, not after it."""
+    w = small_workload(d=128, H_q=16, H_kv=8, b=64, len_lo=3000, len_hi=3000, B=8, n_budget=24, n_local=12)
+    run_fused(w, seed=4, n_app=40, pos_back=64 * 10)
 
 
 FUSED_GATE_CASES = [
