@@ -375,7 +375,6 @@ def test_gate_scores_against_library_matmul():
     for s in range(w.B):
         N = int(c.n_blocks()[s])
         C = N - 1
-        tot = np.zeros(C)
         for qh in range(w.H_q):
             h = qh // w.G
             u = (kg[s, :C, h] @ (Wq @ qf[s, qh])) / math.sqrt(w.dg)
@@ -383,8 +382,6 @@ def test_gate_scores_against_library_matmul():
             np.testing.assert_allclose(logg[s, qh, :C], lg, rtol=1e-12, atol=1e-12)
             assert logg[s, qh, N - 1] == 0.0  # current block B0: unit gate
             assert np.exp(logg[s, qh, :C]).sum() == pytest.approx(1.0, abs=1e-12)
-            if qh % w.G == w.G - 1:
-                tot += 0
         for h in range(w.H_kv):
             g = np.exp(logg[s, h * w.G:(h + 1) * w.G, :C]).sum(0)
             np.testing.assert_allclose(score[s, h, :C], g, rtol=1e-12, atol=1e-14)
