@@ -264,10 +264,11 @@ int sba_score_select_static(const sba_cache *c, const void *q, const sba_select_
 int sba_fold_gate(const sba_gate *gate, float *A, void *stream);
 
 /* Cluster size (CTAs per sequence and KV group) that sba_decode_step uses on
- * the current device for this cache shape and rule: the largest power of two
- * <= 16 with every cluster resident at once when possible (one CTA per SM).
- * Sets kernel attributes, launches nothing; 0 if the shape is not supported
- * by the fused step. */
+ * the current device for this cache shape and rule: the largest C <= 16 with
+ * B * H_kv * C <= the SM count whose clusters are all resident at once (one
+ * CTA per SM), else the largest C the device can schedule.  Remembered per
+ * device and shape.  Sets kernel attributes, launches nothing; 0 if the shape
+ * is not supported by the fused step or no device is present. */
 int32_t sba_decode_step_cluster(const sba_cache *c, const sba_select_params *p);
 
 /* One whole decode step of one layer in ONE launch: rows a1-a6 fused.

@@ -128,3 +128,45 @@ def test_rejects_bad_decode_combine_append_update_on_host():
     g = sba.sba_gate(None, 0x100, 128)
     assert upd(ctypes.byref(c), 0x3000, 1, ctypes.byref(g), None) == E
     assert upd(ctypes.byref(_cache(desc=None)), 0x3000, 1, None, None) == E
+
+
+def _step(c, q=0x5000, k_new=None, v_new=None, pos=None, n_new=0, gate_A=None, p=None, scale=0.088,
+          out=0x9000, out_dtype=0, lse=None, sel=None, cnt=None, gb=None, n_max=0):
+    lib = sba.load()
+    p = p or sba.select_params(16, 2, 0, 0, 0, 0)
+    return lib.sba_decode_step(ctypes.byref(c), q, k_new, v_new, pos, n_new, gate_A, ctypes.byref(p), scale, out,
+                               out_dtype, lse, sel, cnt, gb, n_max, None)
+
+
+def test_rejects_bad_decode_step_arguments_on_host():
+    """The fused step checks its arguments before any device work."""
+    E = sba.SBA_ERR_INVALID_ARG
+    c = _cache()
+    assert _step(_cache(k=None)) == E
+    assert _step(_cache(d=64)) == sba.SBA_ERR_UNSUPPORTED
+    assert _step(c, q=None) == E
+    assert _step(c, q=0x5008) == E                      # q not 16-byte aligned
+    assert _step(c, out=None) == E
+    assert _step(c, out_dtype=7) == E
+    assert _step(c, scale=0.0) == E
+    assert _step(c, scale=float("nan")) == E
+    assert _step(c, n_new=-1) == E
+    assert _step(c, n_new=1, k_new=0x1000, v_new=0x2000) == E                 # no positions
+    assert _step(c, n_new=1, k_new=None, v_new=0x2000, pos=0x3000) == E
+    assert _step(c, n_new=1, k_new=0x1008, v_new=0x2000, pos=0x3000) == E     # misaligned rows
+    assert _step(_cache(desc=None)) == E                                      # Quest needs descriptors
+    gate = sba.select_params(16, 2, 0, 0, 0, 1)
+    assert _step(_cache(kg=0x9000), p=gate) == E                              # gate needs the folded A
+    assert _step(c, p=gate, gate_A=0xa000) == E                               # ... and stored gate keys
+    assert _step(c, sel=0xb000, cnt=0xc000, n_max=15) == E                    # 16 blocks can be selected
+    assert _step(c, p=sba.select_params(16, 2, 0, 5, 4, 0)) == E              # keep fraction > 1
+
+
+def test_rejects_bad_fold_gate_arguments_on_host():
+    lib = sba.load()
+    E = sba.SBA_ERR_INVALID_ARG
+    assert lib.sba_fold_gate(None, 0x1000, None) == E
+    for g in (sba.sba_gate(None, 0x100, 128), sba.sba_gate(0x100, None, 128), sba.sba_gate(0x100, 0x200, 0),
+              sba.sba_gate(0x100, 0x200, 257)):
+        assert lib.sba_fold_gate(ctypes.byref(g), 0x1000, None) == E
+    assert lib.sba_fold_gate(ctypes.byref(sba.sba_gate(0x100, 0x200, 128)), None, None) == E
