@@ -12,9 +12,12 @@ Flash-Decoding, PagedAttention); "SAS: Simple Attention Sparsification via
 End-to-End Optimization of Context Ranking" (Method, Limitations);
 "SeerAttention-R: Sparse Attention Adaptation for Long Reasoning" (abstract).
 
-Parity status of each function is pinned by tests/test_oracle_pins.py; the
-end-to-end numbers are "parity unpinned" against the pages (they print no
-worked example), so correctness rests on those pins.
+Parity status of each function is pinned by tests/test_oracle_pins.py (swept
+by tests/test_oracle_properties.py, guarded by tests/test_oracle_mutations.py);
+the end-to-end numbers are "parity unpinned" against the pages (they print no
+worked example), so correctness rests on those pins.  The modules
+``sas_variants`` and ``multi_query`` extend it to the next rows of the build
+(pinned by their own test files) and have no CUDA counterpart yet.
 """
 from __future__ import annotations
 
