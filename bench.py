@@ -6,7 +6,13 @@ descriptors of the touched blocks, score + select, sparse decode, combine --
 all through libsba's C ABI, captured once in a CUDA graph and replayed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --sweep [--steps K]     # one line per context, R1-7B and Qwen3-14B shapes
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+The default workload is the largest single-GPU one, the Qwen3-14B-shaped gated
+decode at 524288 tokens (40 layers).  The workload with a rectification window
+(R1-7B shape, f = 32) also times the dense rectification pass of all layers and
+reports the step with that pass amortised over f steps.
 
 Multi-GPU (torchrun, one process per GPU): every rank decodes its own
 independent batch of the same shape (weak scaling); no collective touches the
@@ -32,7 +38,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-decode µs/step and achieved HBM GB/s (% of B200 roofline) vs context"
-DEFAULT_WORKLOAD = "qwen3_4b"
+DEFAULT_WORKLOAD = "qwen3_14b_gate"
+SWEEP_SHAPES = ["r1_7b_256k", "qwen3_14b_gate"]
+SWEEP_CONTEXTS = [16384, 32768, 65536, 131072, 262144, 524288]
 DESC_BYTES = 512  # Quest bf16 min+max, or gate fp32 key, per block and KV head
 
 
@@ -50,7 +58,32 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--path", default="fused", choices=["fused", "separate"],
                     help="fused: one sba_decode_step launch per layer; separate: the five single-step calls")
+    ap.add_argument("--context", type=int, default=0, help="override the workload's context length")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per context in SWEEP_CONTEXTS for each shape in SWEEP_SHAPES")
+    ap.add_argument("--cpu-threads", type=int, default=0, help="threads of the all-cores oracle (0 = affinity)")
     return ap.parse_args()
+
+
+def select_params_of(w):
+    """The C selection rule of a workload (scorer, budget, gate position and activation)."""
+    from block_sparse_gqa_min_b200 import sba
+
+    gate = w.scorer == "gate"
+    pos = {"off": sba.SBA_LOG_GATE_OFF, "inner": sba.SBA_LOG_GATE_INNER, "outer": sba.SBA_LOG_GATE_OUTER}
+    act = {"softmax": sba.SBA_GATE_SOFTMAX, "sigmoid": sba.SBA_GATE_SIGMOID, "raw": sba.SBA_GATE_RAW}
+    return sba.select_params(w.n_budget, w.n_local, w.n_min, w.keep_num, w.keep_den,
+                             sba.SBA_SCORER_GATE if gate else sba.SBA_SCORER_QUEST,
+                             pos[w.gate_position] if gate else 0, act[w.gate_act] if gate else 0)
+
+
+def workload_of(args):
+    from block_sparse_gqa_min_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    if args.context:
+        w = w.with_(len_lo=args.context, len_hi=args.context)
+    return w
 
 
 def dist_env():
@@ -205,8 +238,7 @@ def build_layers(w, lay, seed, n_layers, dev):
     from block_sparse_gqa_min_b200 import workloads as W
 
     gate = w.scorer == "gate"
-    p = sba.select_params(w.n_budget, w.n_local, w.n_min, w.keep_num, w.keep_den,
-                          sba.SBA_SCORER_GATE if gate else sba.SBA_SCORER_QUEST)
+    p = select_params_of(w)
     layers = []
     max_len = int(lay.seq_lens.max().item())
     ws = None
@@ -260,9 +292,87 @@ def layer_step(w, L, p, pos, q=None, k_new=None, v_new=None, path="fused", out=N
 KERNELS_PER_LAYER = {"fused": 1, "separate": 5}  # separate: append, update, score+select, decode, combine
 
 
-def native(args, rank, world, local):
+def capture(fn):
+    """One CUDA graph of fn() (after one eager run on a side stream)."""
+    import torch
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fn()
+    torch.cuda.synchronize()
+    return graph
+
+
+def time_graph(graph, steps, warmup, flush_buf, world, local, clocks=True):
+    """Mean device time (ms) of one replay over `steps` replays after `warmup`, CUDA events on
+    the replay stream; a 512 MB write between replays (outside the events) when flush_buf is
+    given.  Returns (ms, clock record)."""
     import torch
     import torch.distributed as dist
+
+    for _ in range(max(warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps + 2)]
+    if flush_buf is not None:
+        for i in range(steps):
+            flush_buf.fill_(float(i))
+            ev[2 * i].record()
+            graph.replay()
+            ev[2 * i + 1].record()
+        torch.cuda.synchronize()
+        total_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps))
+    else:
+        ev[0].record()
+        for _ in range(steps):
+            graph.replay()
+        ev[1].record()
+        torch.cuda.synchronize()
+        total_ms = ev[0].elapsed_time(ev[1])
+    clk = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    return total_ms / steps, clk
+
+
+def append_update_bytes(w, lens):
+    """Bytes a step writes beyond its counted reads (reported apart, per layer): the appended
+    K and V rows, and the refreshed descriptor of every block they touch."""
+    tot = 0
+    for L in lens:
+        p0 = max(int(L) - w.append_tokens, 0)
+        touched = (int(L) - 1) // w.b - p0 // w.b + 1 if L > 0 else 0
+        tot += w.append_tokens * w.H_kv * w.d * 2 * 2 + touched * w.H_kv * DESC_BYTES
+    return tot
+
+
+def rect_bytes(w, lens):
+    """Algorithmic bytes of one rectification pass of one layer: every valid K and V row of the
+    cache read once, the window's rows written, the touched blocks' descriptors written."""
+    f = w.rectify_every
+    tot = 0
+    for L in lens:
+        L = int(L)
+        touched = (L - 1) // w.b - max(L - f, 0) // w.b + 1 if L > 0 else 0
+        tot += L * w.H_kv * w.d * 2 * 2 + f * w.H_kv * w.d * 2 * 2 + touched * w.H_kv * DESC_BYTES
+    return tot
+
+
+def native(args, rank, world, local, w=None, sweep=False):
+    import torch
 
     from block_sparse_gqa_min_b200 import sba
     from block_sparse_gqa_min_b200 import workloads as W
@@ -270,7 +380,7 @@ def native(args, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     sba.load()
-    w = W.WORKLOADS[args.workload]
+    w = w or workload_of(args)
     n_layers = args.layers or w.layers
     seed = rank_seed(args.seed, rank)
     lay = W.make_layout(w, seed, device=dev)
@@ -282,77 +392,73 @@ def native(args, rank, world, local):
     step_bytes = per_layer * n_layers
     kv_bytes_layer = sum(sba.sba_num_selected((L + w.b - 1) // w.b, p) * w.b * w.d * 4 * w.H_kv for L in lens)
     desc_bytes_layer = sum(((L + w.b - 1) // w.b) * w.H_kv * DESC_BYTES for L in lens)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = step_bytes < 4 * l2
+    flush_buf = torch.empty((512 * 1024 * 1024 // 4,), dtype=torch.float32, device=dev) if flush else None
+
+    # ---- the rectification pass (every f steps), timed first: the cache it leaves is the one
+    # the decode step then runs on, and the one the oracle checks below ----
+    rect = None
+    if w.rectify_every and args.path == "fused" and not sweep:
+        f = w.rectify_every
+        rins = [W.make_rect_inputs(w, seed, l, device=dev) for l in range(n_layers)]
+        rg = sba.sba_multi_row_groups(layers[0]["c"], f)
+        N_max = (lay.max_blocks)
+        S_r = max(1, min(N_max, torch.cuda.get_device_properties(dev).multi_processor_count // (w.B * w.H_kv * rg)))
+        o_r = torch.empty((w.B, f, w.H_q, S_r, w.d), dtype=torch.float32, device=dev)
+        l_r = torch.empty((w.B, f, w.H_q, S_r), dtype=torch.float32, device=dev)
+        out_r = torch.empty((w.B, f * w.H_q, w.d), dtype=torch.float32, device=dev)
+        lse_r = torch.empty((w.B, f * w.H_q), dtype=torch.float32, device=dev)
+
+        def rect_pass():
+            for L, ri in zip(layers, rins):
+                sba.sba_rectify(L["c"], ri.q, ri.k_new, ri.v_new, w.scale, o_r, l_r)
+                sba.sba_combine(o_r, l_r, out_r, lse_r)
+
+        rgraph = capture(rect_pass)
+        r_ms, _ = time_graph(rgraph, max(3, min(args.steps, 10)), args.warmup, None, world, local, clocks=False)
+        r_ms = max_over_ranks(r_ms, world, dev)
+        rb = rect_bytes(w, lens) * n_layers
+        hbm, _ = peaks()
+        rect = {"every_steps": f, "us_per_pass": round(r_ms * 1e3, 1), "us_per_layer": round(r_ms * 1e3 / n_layers, 2),
+                "bytes_per_pass": rb, "gbs": round(job_gbs(rb, world, r_ms), 1),
+                "frac_of_measured_hbm": round(job_gbs(rb, 1, r_ms) / hbm, 4),
+                "num_splits": S_r, "row_groups": rg,
+                "kernels": "mq_decode_kernel<dense> + combine_kernel per layer (one CUDA graph)"}
+        del rgraph
 
     def step():
         for L in layers:
             layer_step(w, L, p, pos, path=args.path)
 
-    # capture one step in a CUDA graph
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        step()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    torch.cuda.synchronize()
-
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    footprint = step_bytes
-    flush = footprint < 4 * l2
-    flush_buf = torch.empty((512 * 1024 * 1024 // 4,), dtype=torch.float32, device=dev) if flush else None
-
-    for _ in range(max(args.warmup, 3)):
-        graph.replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps + 2)]
-    if flush:
-        total_ms = 0.0
-        for i in range(args.steps):
-            flush_buf.fill_(float(i))
-            ev[2 * i].record()
-            graph.replay()
-            ev[2 * i + 1].record()
-        torch.cuda.synchronize()
-        total_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps))
-    else:
-        ev[0].record()
-        for _ in range(args.steps):
-            graph.replay()
-        ev[1].record()
-        torch.cuda.synchronize()
-        total_ms = ev[0].elapsed_time(ev[1])
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    ms_max = max_over_ranks(total_ms / args.steps, world, dev)
+    graph = capture(step)
+    ms, clk = time_graph(graph, args.steps, args.warmup, flush_buf, world, local)
+    ms_max = max_over_ranks(ms, world, dev)
     value = job_gbs(step_bytes, world, ms_max)
+    hbm, peak_kind = peaks()
+    step_frac = step_bytes / (ms_max * 1e-3) / 1e9 / hbm
 
-    # ---- per-launch durations, measured live on the launching stream ----
-    # launches are queued behind a sleep kernel so that host-side gaps between
-    # them do not appear in the device-side event intervals
-    names = ["decode_step"] if args.path == "fused" else ["append_kv", "update_descriptors", "score_select",
-                                                          "sparse_decode", "combine"]
-    kt = {k: [] for k in names}
-    for _ in range(3):
-        torch.cuda._sleep(int(2e8))
-        rec = []
-        for L in layers:
-            c, li, bufs = L["c"], L["li"], L["bufs"]
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-            ev[0].record()
-            if args.path == "fused":
-                layer_step(w, L, p, pos, path="fused")
-                ev[1].record()
-            else:
+    # ---- roofline of the dominant kernel ----
+    if args.path == "fused":
+        # one launch per layer inside the graph: its in-step duration is the step time over the
+        # launches (consecutive layers overlap only by programmatic-dependent-launch prologues)
+        launch_ms = ms_max / n_layers
+        achieved = per_layer / (launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "decode_step", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": peak_kind, "alg_bytes_per_launch": per_layer,
+                "launch_us": round(launch_ms * 1e3, 3),
+                "launch_us_source": "graph-replayed step time / launches per step (CUDA events)",
+                "traffic": recorded_traffic("decode_step", w.name), "step_frac": round(step_frac, 4)}
+    else:
+        names = ["append_kv", "update_descriptors", "score_select", "sparse_decode", "combine"]
+        kt = {k: [] for k in names}
+        for _ in range(3):
+            torch.cuda._sleep(int(2e8))
+            rec = []
+            for L in layers:
+                c, li, bufs = L["c"], L["li"], L["bufs"]
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+                ev[0].record()
                 sba.sba_append_kv(c, li.k_new, li.v_new, pos)
                 ev[1].record()
                 if w.scorer == "gate":
@@ -367,29 +473,26 @@ def native(args, rank, world, local):
                 ev[4].record()
                 sba.sba_combine(bufs.o_part, bufs.lse_part, bufs.out, bufs.lse)
                 ev[5].record()
-            rec.append(ev)
-        torch.cuda.synchronize()
-        for ev in rec:
-            for i, k in enumerate(names):
-                kt[k].append(ev[i].elapsed_time(ev[i + 1]))
-    kmean = {k: statistics.mean(v) for k, v in kt.items()}
-    if args.path == "fused":
-        alg = {"decode_step": per_layer}
-    else:
+                rec.append(ev)
+            torch.cuda.synchronize()
+            for ev in rec:
+                for i, k in enumerate(names):
+                    kt[k].append(ev[i].elapsed_time(ev[i + 1]))
+        kmean = {k: statistics.mean(v) for k, v in kt.items()}
         alg = {"sparse_decode": kv_bytes_layer, "score_select": desc_bytes_layer}
-    dom = max(alg, key=lambda k: kmean[k])
-    hbm, peak_kind = peaks()
-    achieved = alg[dom] / (kmean[dom] * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-            "frac": round(achieved / hbm, 4), "peak_source": peak_kind,
-            "alg_bytes_per_launch": alg[dom], "launch_us": round(kmean[dom] * 1e3, 3),
-            "traffic": recorded_traffic(dom, w.name),
-            "other_kernels_us": {k: round(v * 1e3, 3) for k, v in kmean.items() if k != dom},
-            "step_frac": round(step_bytes / (ms_max * 1e-3) / 1e9 / hbm, 4)}
+        dom = max(alg, key=lambda k: kmean[k])
+        achieved = alg[dom] / (kmean[dom] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "peak_source": peak_kind, "alg_bytes_per_launch": alg[dom],
+                "launch_us": round(kmean[dom] * 1e3, 3),
+                "launch_us_source": "eager launches behind a sleep kernel (CUDA events)",
+                "traffic": recorded_traffic(dom, w.name),
+                "other_kernels_us": {k: round(v * 1e3, 3) for k, v in kmean.items() if k != dom},
+                "step_frac": round(step_frac, 4)}
 
     # ---- e2e: host buffers, copies inside the timed region ----
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not sweep:
         # a step's inputs of every layer in one pinned host buffer per tensor, every layer's output
         # back in one copy: one host-to-device copy per input tensor and one device-to-host copy
         def stacked(ts):
@@ -422,6 +525,8 @@ def native(args, rank, world, local):
             e2e_step()
         torch.cuda.synchronize()
         if world > 1:
+            import torch.distributed as dist
+
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, min(args.steps, 20))
@@ -436,13 +541,17 @@ def native(args, rank, world, local):
                "api": ("eager C-ABI call per layer; q, k_new, v_new of all layers from one pinned host buffer "
                        "each (one copy per tensor per step), every layer's fp32 output back in one copy")}
 
+    # the graph's last replay left the selection of every layer in its buffers (same inputs every
+    # replay); the status words must be clean
+    graph.replay()
+    torch.cuda.synchronize()
     status = [int(L["c"].status.item()) for L in layers]
     if any(status):
         raise RuntimeError(f"device status bits set: {status}")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, lay, layers, p, args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not sweep:
+        cpu = cpu_baseline(w, lay, layers, p, args.cpu_seconds, args.cpu_threads)
 
     out = {
         "metric": METRIC,
@@ -453,6 +562,7 @@ def native(args, rank, world, local):
         "warmup": max(args.warmup, 3),
         "ms_per_step": round(ms_max, 4),
         "us_per_step": round(ms_max * 1e3, 1),
+        "us_per_layer": round(ms_max * 1e3 / n_layers, 2),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -462,12 +572,15 @@ def native(args, rank, world, local):
             "workload": w.name, "batch": w.B, "layers": n_layers, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
             "block": w.b, "context": [min(lens), max(lens)], "blocks_selected_per_group": n_max,
             "scorer": w.scorer, "paged": w.paged, "append_tokens_per_step": w.append_tokens,
+            "log_gate": w.gate_position if w.scorer == "gate" else None,
+            "gate_act": w.gate_act if w.scorer == "gate" else None,
             "num_splits": splits, "cluster_ctas": sba.sba_decode_step_cluster(layers[0]["c"], p),
             "counted_bytes_per_step": step_bytes,
             "kv_bytes_per_layer": kv_bytes_layer, "desc_bytes_per_layer": desc_bytes_layer,
+            "append_update_bytes_per_layer": append_update_bytes(w, lens),
             "l2": (f"L2 flushed between steps (512 MB write, outside the timed events); step footprint "
-                   f"{footprint / 1e6:.0f} MB" if flush else
-                   f"inputs larger than L2: {footprint / 1e6:.0f} MB per step vs {l2 / 1e6:.0f} MB L2"),
+                   f"{step_bytes / 1e6:.0f} MB" if flush else
+                   f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step vs {l2 / 1e6:.0f} MB L2"),
             "graph": "one CUDA graph per step, programmatic dependent launch between kernels",
             "path": ("one fused sba_decode_step launch per layer (thread-block clusters)" if args.path == "fused"
                      else "five C-ABI calls per layer"),
@@ -479,6 +592,13 @@ def native(args, rank, world, local):
         "gpu_launches": KERNELS_PER_LAYER[args.path] * n_layers * args.steps,
         "clocks": clk,
     }
+    if rect is not None:
+        f = rect["every_steps"]
+        amort_ms = ms_max + rect["us_per_pass"] * 1e-3 / f
+        rect["step_with_pass_amortised"] = {
+            "us_per_step": round(amort_ms * 1e3, 1),
+            "gbs": round(job_gbs(step_bytes + rect["bytes_per_pass"] / f, world, amort_ms), 1)}
+        out["rectify"] = rect
     del graph
     return out
 
@@ -487,7 +607,13 @@ def native(args, rank, world, local):
 # CPU oracle (timed baseline and the --impl reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(w, lay_cpu, layer_inputs_fn, n_layers, budget_s, p_num_sel):
+def _oracle_kwargs(w):
+    kw = dict(scale=w.scale, n_budget=w.n_budget, n_local=w.n_local, n_min=w.n_min, keep_num=w.keep_num,
+              keep_den=w.keep_den, scorer=w.scorer, log_gate=w.gate_position != "off")
+    return kw
+
+
+def oracle_sample(w, lay_cpu, layer_inputs_fn, n_layers, budget_s, p_num_sel, on_result=None):
     """Run the oracle's whole step (descriptors -> scores -> selection ->
     attention) on evenly spaced layers until `budget_s` seconds are used."""
     import oracle as O
@@ -503,14 +629,15 @@ def oracle_sample(w, lay_cpu, layer_inputs_fn, n_layers, budget_s, p_num_sel):
         oc = O.Cache(W.bf16_bits(li.k), W.bf16_bits(li.v),
                      None if lay_cpu.block_table is None else lay_cpu.block_table.numpy(),
                      lay_cpu.seq_lens.numpy(), H_q=w.H_q, max_blocks=lay_cpu.max_blocks)
-        kw = dict(scale=w.scale, n_budget=w.n_budget, n_local=w.n_local, n_min=w.n_min, keep_num=w.keep_num,
-                  keep_den=w.keep_den, scorer=w.scorer)
+        kw = _oracle_kwargs(w)
         if w.scorer == "gate":
             kw.update(Wq=li.Wq.cpu().numpy(), Wk=li.Wk.cpu().numpy())
         qb = W.bf16_bits(li.q)
         t0 = time.perf_counter()
-        O.decode(oc, qb, **kw)
+        res = O.decode(oc, qb, **kw)
         t_cpu += time.perf_counter() - t0
+        if on_result is not None:
+            on_result(l, res)
         done.append(l)
         bytes_done += per_layer
         if t_cpu >= budget_s:
@@ -518,37 +645,121 @@ def oracle_sample(w, lay_cpu, layer_inputs_fn, n_layers, budget_s, p_num_sel):
     return done, t_cpu, bytes_done
 
 
-def cpu_baseline(w, lay, layers, p, budget_s):
+def oracle_all_cores(w, lay_cpu, layer_inputs_fn, n_layers, budget_s, p_num_sel, threads):
+    """The same oracle, unchanged, run as independent (layer, sequence, KV group) problems on a
+    pool of `threads` threads (the C oracle runs outside the GIL): each problem is the layer's
+    cache restricted to one KV head and its G query heads.  Whole layers are taken, in the
+    single-threaded sample's order, until about `budget_s` seconds of wall time are used."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import oracle as O
+    from block_sparse_gqa_min_b200 import workloads as W
+
+    order = sorted(set([0, n_layers - 1, n_layers // 2] + list(range(n_layers))), key=lambda l: (
+        0 if l in (0, n_layers - 1, n_layers // 2) else 1, l))
+    lens = lay_cpu.seq_lens.tolist()
+    per_layer = counted_bytes(w, lens, p_num_sel)
+    bt = None if lay_cpu.block_table is None else lay_cpu.block_table.numpy()
+    G = w.G
+    t_wall, done, nbytes = 0.0, [], 0
+    with ThreadPoolExecutor(max_workers=threads) as pool:
+        for l in order:
+            li = layer_inputs_fn(l)
+            kb, vb, qb = W.bf16_bits(li.k), W.bf16_bits(li.v), W.bf16_bits(li.q)
+            jobs = []
+            for h in range(w.H_kv):  # (the whole batch per head: sequences stay independent inside the oracle)
+                oc = O.Cache(np.ascontiguousarray(kb[:, h:h + 1]), np.ascontiguousarray(vb[:, h:h + 1]), bt,
+                             lay_cpu.seq_lens.numpy(), H_q=G, max_blocks=lay_cpu.max_blocks)
+                kw = _oracle_kwargs(w)
+                if w.scorer == "gate":
+                    kw.update(Wq=li.Wq.cpu().numpy(), Wk=li.Wk.cpu().numpy())
+                jobs.append((oc, np.ascontiguousarray(qb[:, h * G:(h + 1) * G]), kw))
+            t0 = time.perf_counter()
+            list(pool.map(lambda j: O.decode(j[0], j[1], **j[2]), jobs))
+            t_wall += time.perf_counter() - t0
+            done.append(l)
+            nbytes += per_layer
+            if t_wall >= budget_s:
+                break
+    return done, t_wall, nbytes
+
+
+def cpu_baseline(w, lay, layers, p, budget_s, threads=0):
+    """The oracle timed on this host: all cores (threads over independent KV groups) as the
+    reported baseline, single-threaded beside it; the sampled layers' oracle selections are
+    compared with the GPU's (exact, near-tie within 1e-5 relative, or mismatch)."""
+    import numpy as np
+
     from block_sparse_gqa_min_b200 import sba
     from block_sparse_gqa_min_b200 import workloads as W
 
     lay_cpu = W.Layout(lay.seq_lens.cpu(), None if lay.block_table is None else lay.block_table.cpu(),
                        lay.num_pages, lay.max_blocks)
+    cache = {}
 
     def fn(l):
-        li = layers[l]["li"]
-        return W.LayerInputs(li.q.cpu(), li.k.cpu(), li.v.cpu(), li.k_new, li.v_new,
-                             None if li.Wq is None else li.Wq.cpu(), None if li.Wk is None else li.Wk.cpu())
+        if l not in cache:
+            cache.clear()
+            li = layers[l]["li"]
+            cache[l] = W.LayerInputs(li.q.cpu(), li.k.cpu(), li.v.cpu(), li.k_new, li.v_new,
+                                     None if li.Wq is None else li.Wq.cpu(), None if li.Wk is None else li.Wk.cpu())
+        return cache[l]
 
-    done, t, nbytes = oracle_sample(w, lay_cpu, fn, len(layers), budget_s, lambda N: sba.sba_num_selected(N, p))
-    return {"value": round(nbytes / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seconds": round(t, 2), "us_per_step_equiv": round(t / len(done) * len(layers) * 1e6, 1),
-            "sample": (f"{len(done)} of {len(layers)} layers (whole layer each: descriptors, scores, selection, "
-                       f"fp64 attention), single-threaded C oracle; excludes host copies")}
+    sel_check = {"layers": 0, "groups": 0, "exact": 0, "near_tie_events": 0, "mismatch": 0}
+    L_eff = max(w.n_local, 1) if w.scorer == "gate" else w.n_local
+
+    def compare(l, ref):
+        gi = layers[l]["bufs"].sel_idx.cpu().numpy()
+        gc = layers[l]["bufs"].sel_cnt.cpu().numpy()
+        sel_check["layers"] += 1
+        N_all = ((lay_cpu.seq_lens.numpy().astype(np.int64) + w.b - 1) // w.b)
+        for s in range(w.B):
+            N = int(N_all[s])
+            Lc = min(L_eff, N)
+            for h in range(w.H_kv):
+                sel_check["groups"] += 1
+                n = int(ref.sel_cnt[s, h])
+                a, b = set(ref.sel_idx[s, h, :n].tolist()), set(gi[s, h, :int(gc[s, h])].tolist())
+                if int(gc[s, h]) == n and a == b:
+                    sel_check["exact"] += 1
+                    continue
+                sc = ref.score[s, h, : N - Lc].astype(np.float32).astype(np.float64)
+                adm = [j for j in a if j < N - Lc]
+                theta = min(sc[j] for j in adm) if adm else 0.0
+                ok = int(gc[s, h]) == n and all(j < N - Lc and abs(sc[j] - theta) <= 1e-5 * abs(theta)
+                                                for j in a.symmetric_difference(b))
+                sel_check["near_tie_events" if ok else "mismatch"] += 1
+
+    num_sel = lambda N: sba.sba_num_selected(N, p)  # noqa: E731
+    done1, t1, nb1 = oracle_sample(w, lay_cpu, fn, len(layers), budget_s, num_sel, on_result=compare)
+    threads = threads or len(os.sched_getaffinity(0))
+    doneN, tN, nbN = oracle_all_cores(w, lay_cpu, fn, len(layers), budget_s, num_sel, threads)
+    return {"value": round(nbN / tN / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": round(tN, 2), "us_per_step_equiv": round(tN / len(doneN) * len(layers) * 1e6, 1),
+            "sample": (f"{len(doneN)} of {len(layers)} layers (whole layers: descriptors, scores, selection, fp64 "
+                       f"attention), the unchanged C oracle run as independent KV-group problems on {threads} "
+                       f"threads; excludes host copies"),
+            "single_core": {"value": round(nb1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                            "seconds": round(t1, 2), "us_per_step_equiv": round(t1 / len(done1) * len(layers) * 1e6, 1),
+                            "sample": f"{len(done1)} of {len(layers)} whole layers, single-threaded C oracle"},
+            "selection_check": sel_check}
 
 
 def reference(args, rank, world):
-    """The oracle as the reference arm, on this host's cores."""
+    """The oracle as the reference arm, on this host's cores: every step is a bounded sample of
+    the workload's layers, run as independent KV-group problems on all the cores this process
+    may use."""
     if rank != 0:
         return None
-    import numpy as np  # noqa: F401
     import torch
 
     import oracle as O
     from block_sparse_gqa_min_b200 import workloads as W
 
     O.build()
-    w = W.WORKLOADS[args.workload]
+    w = workload_of(args)
     n_layers = args.layers or w.layers
     lay = W.make_layout(w, args.seed, device="cpu")
 
@@ -564,12 +775,13 @@ def reference(args, rank, world):
             cache[l] = W.make_layer(w, lay, args.seed, l, device="cpu")
         return cache[l]
 
+    threads = args.cpu_threads or len(os.sched_getaffinity(0))
     per_step_budget = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(w, lay, fn, n_layers, 0.0, num_sel)
+        oracle_all_cores(w, lay, fn, n_layers, 0.0, num_sel, threads)
     times, nbytes_all, layers_all = [], 0, 0
     for _ in range(args.steps):
-        done, t, nb = oracle_sample(w, lay, fn, n_layers, per_step_budget, num_sel)
+        done, t, nb = oracle_all_cores(w, lay, fn, n_layers, per_step_budget, num_sel, threads)
         times.append(t)
         nbytes_all += nb
         layers_all += len(done)
@@ -577,16 +789,19 @@ def reference(args, rank, world):
     value = nbytes_all / tot / 1e9
     ms_step = tot / layers_all * n_layers * 1e3
     torch.set_num_threads(1)
+    lens = lay.seq_lens.tolist()
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "us_per_step": round(ms_step * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded)",
-        "config": {"workload": w.name, "batch": w.B, "layers": n_layers, "H_q": w.H_q, "H_kv": w.H_kv,
-                   "block": w.b, "context": [int(lay.seq_lens.min()), int(lay.seq_lens.max())]},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{layers_all} layer-passes over {args.steps} steps (whole layers, "
-                                   f"single-threaded C oracle, fp64)"},
+        "data": "synthetic (seeded; shapes and distributions of the workload, no model weights)",
+        "config": {"workload": w.name, "batch": w.B, "layers": n_layers, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
+                   "block": w.b, "context": [min(lens), max(lens)], "scorer": w.scorer, "paged": w.paged},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{layers_all} layer-passes over {args.steps} steps (whole layers, the "
+                                   f"unchanged C oracle in fp64 as independent KV-group problems on {threads} "
+                                   f"threads)"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -616,9 +831,22 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
-    out = native(args, rank, world, local)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
+    if args.sweep:
+        # the "vs context" curve: every context at the R1-7B and Qwen3-14B shapes, one line each
+        from block_sparse_gqa_min_b200 import workloads as W
+
+        for shape in SWEEP_SHAPES:
+            for ctx in SWEEP_CONTEXTS:
+                w = W.WORKLOADS[shape].with_(len_lo=ctx, len_hi=ctx)
+                out = native(args, rank, world, local, w=w, sweep=True)
+                out["config"]["sweep"] = f"{shape} shape at context {ctx}"
+                if rank == 0:
+                    print(json.dumps(out), flush=True)
+                torch.cuda.empty_cache()
+    else:
+        out = native(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -45,8 +45,33 @@ int check_params(const sba_select_params* p) {
     if (p->keep_den < 0 || p->keep_num < 0 || (p->keep_den > 0 && p->keep_num > p->keep_den))
         return SBA_ERR_INVALID_ARG;
     if (p->scorer != SBA_SCORER_QUEST && p->scorer != SBA_SCORER_GATE) return SBA_ERR_INVALID_ARG;
+    if (p->log_gate < SBA_LOG_GATE_OFF || p->log_gate > SBA_LOG_GATE_OUTER) return SBA_ERR_INVALID_ARG;
+    if (p->gate_act < SBA_GATE_SOFTMAX || p->gate_act > SBA_GATE_RAW) return SBA_ERR_INVALID_ARG;
+    if (p->scorer == SBA_SCORER_QUEST && (p->log_gate != 0 || p->gate_act != 0)) return SBA_ERR_INVALID_ARG;
     return SBA_OK;
 }
+
+}  // namespace
+
+namespace sba {
+// Every host-side check of sba_score_select except the workspace (also used by the
+// allocation-free variant, which must reject a call before it enqueues anything).
+int check_score_select(const sba_cache* c, const void* q, const sba_select_params* p, const int32_t* sel_idx,
+                       const int32_t* sel_cnt, int32_t n_max) {
+    int rc = check_cache(c);
+    if (rc != SBA_OK) return rc;
+    rc = check_params(p);
+    if (rc != SBA_OK) return rc;
+    if (!q || !sel_idx || !sel_cnt || n_max < 1 || !aligned16(q)) return SBA_ERR_INVALID_ARG;
+    if (p->scorer == SBA_SCORER_QUEST && !c->desc) return SBA_ERR_INVALID_ARG;
+    if (p->scorer == SBA_SCORER_GATE && !c->kg) return SBA_ERR_INVALID_ARG;
+    const int n_need = num_selected((c->max_len + c->b - 1) / c->b, *p);
+    if (n_max < n_need) return SBA_ERR_INVALID_ARG;
+    return SBA_OK;
+}
+}  // namespace sba
+
+namespace {
 
 int after_launch(int rc) {
     if (rc != SBA_OK) return rc;
@@ -124,31 +149,89 @@ int sba_update_descriptors(const sba_cache* c, const int32_t* pos_start, int32_t
 
 int sba_score_select(const sba_cache* c, const void* q, const sba_select_params* p, int32_t* sel_idx,
                      int32_t* sel_cnt, float* gate_bias, int32_t n_max, void* ws, size_t ws_bytes, void* stream) {
-    int rc = check_cache(c);
+    const int rc = check_score_select(c, q, p, sel_idx, sel_cnt, n_max);
     if (rc != SBA_OK) return rc;
-    rc = check_params(p);
-    if (rc != SBA_OK) return rc;
-    if (!q || !sel_idx || !sel_cnt || n_max < 1 || !aligned16(q)) return SBA_ERR_INVALID_ARG;
-    if (p->scorer == SBA_SCORER_QUEST && !c->desc) return SBA_ERR_INVALID_ARG;
-    if (p->scorer == SBA_SCORER_GATE && !c->kg) return SBA_ERR_INVALID_ARG;
-    const int n_need = num_selected((c->max_len + c->b - 1) / c->b, *p);
-    if (n_max < n_need) return SBA_ERR_INVALID_ARG;
     if (!ws || !aligned16(ws) || ws_bytes < score_workspace_bytes(*c, *p)) return SBA_ERR_WORKSPACE;
-    return after_launch(launch_score_select(*c, q, *p, sel_idx, sel_cnt, p->scorer == SBA_SCORER_GATE ? gate_bias : nullptr,
+    return after_launch(launch_score_select(*c, q, 1, *p, sel_idx, sel_cnt, p->scorer == SBA_SCORER_GATE ? gate_bias : nullptr,
                                             n_max, ws, static_cast<cudaStream_t>(stream)));
 }
 
-int sba_sparse_decode(const sba_cache* c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
-                      const float* gate_bias, int32_t n_max, float softmax_scale, int32_t num_splits, float* o_part,
-                      float* lse_part, void* stream) {
+static int sparse_decode_any(const sba_cache* c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
+                             const float* gate_bias, int32_t n_max, float softmax_scale, int32_t num_splits,
+                             float* o_part, float* lse_part, bool outer, void* stream) {
     int rc = check_cache(c);
     if (rc != SBA_OK) return rc;
     if (!q || !sel_idx || !sel_cnt || !o_part || !lse_part || n_max < 1) return SBA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(o_part)) return SBA_ERR_INVALID_ARG;
     if (num_splits < 1 || num_splits > 65535) return SBA_ERR_INVALID_ARG;
     if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return SBA_ERR_INVALID_ARG;
+    if (outer && !gate_bias) return SBA_ERR_INVALID_ARG;
     return after_launch(launch_sparse_decode(*c, q, sel_idx, sel_cnt, gate_bias, n_max, softmax_scale, num_splits,
-                                             o_part, lse_part, static_cast<cudaStream_t>(stream)));
+                                             o_part, lse_part, outer, static_cast<cudaStream_t>(stream)));
+}
+
+int sba_sparse_decode(const sba_cache* c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
+                      const float* gate_bias, int32_t n_max, float softmax_scale, int32_t num_splits, float* o_part,
+                      float* lse_part, void* stream) {
+    return sparse_decode_any(c, q, sel_idx, sel_cnt, gate_bias, n_max, softmax_scale, num_splits, o_part, lse_part,
+                             false, stream);
+}
+
+int sba_sparse_decode_outer(const sba_cache* c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
+                            const float* gate_bias, int32_t n_max, float softmax_scale, int32_t num_splits,
+                            float* o_part, float* lse_part, void* stream) {
+    return sparse_decode_any(c, q, sel_idx, sel_cnt, gate_bias, n_max, softmax_scale, num_splits, o_part, lse_part,
+                             true, stream);
+}
+
+int sba_score_select_multi(const sba_cache* c, const void* q, int32_t M, const sba_select_params* p,
+                           int32_t* sel_idx, int32_t* sel_cnt, int32_t n_max, void* ws, size_t ws_bytes,
+                           void* stream) {
+    const int rc = check_score_select(c, q, p, sel_idx, sel_cnt, n_max);
+    if (rc != SBA_OK) return rc;
+    if (M < 1 || M > kMaxQueryTokens) return SBA_ERR_INVALID_ARG;
+    if (p->scorer != SBA_SCORER_QUEST) return SBA_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws) || ws_bytes < score_workspace_bytes(*c, *p)) return SBA_ERR_WORKSPACE;
+    return after_launch(launch_score_select(*c, q, M, *p, sel_idx, sel_cnt, nullptr, n_max, ws,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+static int check_multi(const sba_cache* c, const void* q, int32_t M, float softmax_scale, int32_t num_splits,
+                       const float* o_part, const float* lse_part) {
+    const int rc = check_cache(c);
+    if (rc != SBA_OK) return rc;
+    if (!q || !o_part || !lse_part || !aligned16(q)) return SBA_ERR_INVALID_ARG;
+    if (M < 1 || M > kMaxQueryTokens) return SBA_ERR_INVALID_ARG;
+    if (num_splits < 1 || num_splits > 65535) return SBA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return SBA_ERR_INVALID_ARG;
+    if ((int64_t)c->H_kv * mq_row_groups(*c, M) > 65535 || c->B > 65535) return SBA_ERR_UNSUPPORTED;
+    return SBA_OK;
+}
+
+int32_t sba_multi_row_groups(const sba_cache* c, int32_t M) {
+    if (check_cache(c) != SBA_OK || M < 1) return 0;
+    return mq_row_groups(*c, M);
+}
+
+int sba_sparse_decode_multi(const sba_cache* c, const void* q, int32_t M, const int32_t* sel_idx,
+                            const int32_t* sel_cnt, int32_t n_max, float softmax_scale, int32_t num_splits,
+                            float* o_part, float* lse_part, void* stream) {
+    const int rc = check_multi(c, q, M, softmax_scale, num_splits, o_part, lse_part);
+    if (rc != SBA_OK) return rc;
+    if (!sel_idx || !sel_cnt || n_max < 1) return SBA_ERR_INVALID_ARG;
+    return after_launch(launch_multi_query(*c, q, M, sel_idx, sel_cnt, n_max, nullptr, nullptr, false,
+                                           softmax_scale, num_splits, o_part, lse_part,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int sba_rectify(const sba_cache* c, const void* q, const void* k_new, const void* v_new, int32_t f,
+                float softmax_scale, int32_t num_splits, float* o_part, float* lse_part, void* stream) {
+    const int rc = check_multi(c, q, f, softmax_scale, num_splits, o_part, lse_part);
+    if (rc != SBA_OK) return rc;
+    if (f > kMaxRectifyTokens) return SBA_ERR_UNSUPPORTED;
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SBA_ERR_INVALID_ARG;
+    return after_launch(launch_multi_query(*c, q, f, nullptr, nullptr, 0, k_new, v_new, true, softmax_scale,
+                                           num_splits, o_part, lse_part, static_cast<cudaStream_t>(stream)));
 }
 
 int sba_combine(const float* o_part, const float* lse_part, int32_t B, int32_t H_q, int32_t num_splits, int32_t d,

@@ -12,6 +12,8 @@ namespace sba {
 constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 16;
 constexpr int kMaxBlocksPerSeq = 32768;  // selection keys live in shared memory
+constexpr int kMaxQueryTokens = 1024;   // query tokens per sequence of the multi-token calls
+constexpr int kMaxRectifyTokens = 128;  // rectification window: its blocks stay in the staging ring
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bounded waits give up after ~2 s
 
 // ---------------------------------------------------------------------------
@@ -27,6 +29,20 @@ __device__ __forceinline__ uint32_t orderable_key(float f) {
     f = f + 0.0f;
     uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// log g of a historical block from its gate logit u ("SAS ...", Method, and the activations
+// of its ablations): softmax u - LSE; unnormalised u (pass lse = 0); sigmoid
+// log(1 / (1 + exp(-u))), written without overflow on either side.
+__device__ __forceinline__ float log_gate_of(float u, float lse, int act) {
+    if (act != SBA_GATE_SIGMOID) return u - lse;
+    return fminf(u, 0.f) - log1pf(expf(-fabsf(u)));
+}
+
+// The gate g itself, as the group's ranking sums it: exp(u - lse) (softmax, raw with lse = 0)
+// or 1 / (1 + exp(-u)) (sigmoid).
+__device__ __forceinline__ float gate_of(float u, float lse, int act) {
+    return act == SBA_GATE_SIGMOID ? 1.f / (1.f + expf(-u)) : expf(u - lse);
 }
 
 __device__ __forceinline__ void report(int32_t* status, int bit) {

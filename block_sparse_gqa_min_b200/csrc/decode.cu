@@ -1,4 +1,5 @@
 // Split-KV sparse decode over the selected blocks, and the split merge.
+// (kOuter: the SAS gate on the values instead of inside the softmax.)
 //
 // "Rectified Sparse Attention for Efficient Long-Sequence Generation",
 // Summary: exact attention over the group's selected blocks only; its
@@ -63,7 +64,7 @@ struct Smem {
     static constexpr int kBytes = kStages * kStage + kMerge + kBars + 1024;  // + alignment slack
 };
 
-template <int kBlk>
+template <int kBlk, bool kOuter>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          DecodeArgs a) {
@@ -176,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (inf.ok) {
                 const float g0 = bias_r ? __ldg(bias_r + i) * kLog2e : 0.f;
                 const float g1 = bias_r8 ? __ldg(bias_r8 + i) * kLog2e : 0.f;
-                decode_block<kBlk>(dst, qa, dyn + st * S::kStage, inf.valid, g0, g1, a.scale_log2, warp, lane);  // slot = warp
+                decode_block<kBlk, kOuter>(dst, qa, dyn + st * S::kStage, inf.valid, g0, g1, a.scale_log2, warp,
+                                           lane);  // slot = warp
             }
             // release the stage (generic-proxy writes ordered before the next TMA write)
             fence_proxy_async_smem();
@@ -274,22 +276,22 @@ bool make_desc_tmap(CUtensorMap* m, void* base, uint64_t pages, int H_kv, int ro
 
 namespace {
 
-template <int kBlk>
+template <int kBlk, bool kOuter>
 int launch_decode_blk(const sba_cache& c, const DecodeArgs& a, cudaStream_t stream) {
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
     if (!make_kv_tmap(&tk, c.k, rows, kBlk) || !make_kv_tmap(&tv, c.v, rows, kBlk)) return SBA_ERR_CUDA;
     const int smem = Smem<kBlk>::kBytes;
-    if (allow_smem<sparse_decode_kernel<kBlk>>(smem) != SBA_OK) return SBA_ERR_CUDA;
+    if (allow_smem<sparse_decode_kernel<kBlk, kOuter>>(smem) != SBA_OK) return SBA_ERR_CUDA;
     dim3 grid(a.num_splits, c.H_kv, c.B);
-    return launch(sparse_decode_kernel<kBlk>, grid, dim3(kThreads), smem, stream, tk, tv, a);
+    return launch(sparse_decode_kernel<kBlk, kOuter>, grid, dim3(kThreads), smem, stream, tk, tv, a);
 }
 
 }  // namespace
 
 int launch_sparse_decode(const sba_cache& c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
                          const float* gate_bias, int n_max, float scale, int num_splits, float* o_part,
-                         float* lse_part, cudaStream_t stream) {
+                         float* lse_part, bool outer, cudaStream_t stream) {
     DecodeArgs a{};
     a.seq_lens = c.seq_lens;
     a.block_table = c.block_table;
@@ -307,7 +309,8 @@ int launch_sparse_decode(const sba_cache& c, const void* q, const int32_t* sel_i
     a.num_splits = num_splits;
     a.o_part = o_part;
     a.lse_part = lse_part;
-    return c.b == 64 ? launch_decode_blk<64>(c, a, stream) : launch_decode_blk<128>(c, a, stream);
+    if (outer) return c.b == 64 ? launch_decode_blk<64, true>(c, a, stream) : launch_decode_blk<128, true>(c, a, stream);
+    return c.b == 64 ? launch_decode_blk<64, false>(c, a, stream) : launch_decode_blk<128, false>(c, a, stream);
 }
 
 int launch_combine(const float* o_part, const float* lse_part, int B, int H_q, int S, void* out, int out_dtype,

@@ -65,8 +65,10 @@ __device__ __forceinline__ void load_q_frags(uint32_t (&qa)[8][4], const __nv_bf
 
 // One staged block: the T tokens of token slot `slot` (0..3).  `stage` is the generic pointer of
 // the stage, `valid` the block's valid token count, g0/g1 the log-gates of
-// rows r and r+8 (already in log2 units).
-template <int kBlk>
+// rows r and r+8 (already in log2 units): added to the logits, or with kOuter
+// ("SAS ...", Method: the gate outside the softmax) left out of the logits and
+// instead multiplied, as g = 2^g, into the weights of the values.
+template <int kBlk, bool kOuter = false>
 __device__ __forceinline__ void decode_block(DecodeState& st, const uint32_t (&qa)[8][4], uint8_t* stage, int valid,
                                              float g0, float g1, float scale_log2, int slot, int lane) {
     using TG = TileGeom<kBlk>;
@@ -102,15 +104,16 @@ __device__ __forceinline__ void decode_block(DecodeState& st, const uint32_t (&q
         }
     }
     // ---- scale, log-gate, mask, online softmax (base 2) ----
+    const float b0 = kOuter ? 0.f : g0, b1 = kOuter ? 0.f : g1;
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int t = tok0 + nt * 8 + cq;
         const bool v0 = t < valid, v1 = t + 1 < valid;
-        sc[nt][0] = v0 ? fmaf(sc[nt][0], scale_log2, g0) : -INFINITY;
-        sc[nt][1] = v1 ? fmaf(sc[nt][1], scale_log2, g0) : -INFINITY;
-        sc[nt][2] = v0 ? fmaf(sc[nt][2], scale_log2, g1) : -INFINITY;
-        sc[nt][3] = v1 ? fmaf(sc[nt][3], scale_log2, g1) : -INFINITY;
+        sc[nt][0] = v0 ? fmaf(sc[nt][0], scale_log2, b0) : -INFINITY;
+        sc[nt][1] = v1 ? fmaf(sc[nt][1], scale_log2, b0) : -INFINITY;
+        sc[nt][2] = v0 ? fmaf(sc[nt][2], scale_log2, b1) : -INFINITY;
+        sc[nt][3] = v1 ? fmaf(sc[nt][3], scale_log2, b1) : -INFINITY;
         mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
         mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
     }
@@ -142,6 +145,16 @@ __device__ __forceinline__ void decode_block(DecodeState& st, const uint32_t (&q
         sc[nt][3] = exp2f(sc[nt][3] - u1);
         st.l0 += sc[nt][0] + sc[nt][1];
         st.l1 += sc[nt][2] + sc[nt][3];
+    }
+    if (kOuter) {  // the block's gate weights its values, not its share of the normaliser
+        const float gm0 = exp2f(g0), gm1 = exp2f(g1);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            sc[nt][0] *= gm0;
+            sc[nt][1] *= gm0;
+            sc[nt][2] *= gm1;
+            sc[nt][3] *= gm1;
+        }
     }
     // ---- O += P V (P as bf16 hi + lo) ----
 #pragma unroll
@@ -263,11 +276,13 @@ __device__ __forceinline__ void load_q_frags_t(uint32_t (&qb)[NH][8][2], const _
 }
 
 // One 64-token stage: the 16 tokens of token slot `slot` (0..3).  gb[nh][x] is the log-gate
-// (log2 units) of head 8nh + 2(lane%4) + x; `valid` counts the stage's valid tokens.
+// (log2 units) of head 8nh + 2(lane%4) + x, added to the logits; with `outer` ("SAS ...",
+// Method: the gate outside the softmax) it stays out of the logits and 2^gb instead weights
+// the values.  `valid` counts the stage's valid tokens.
 template <int NH>
 __device__ __forceinline__ void decode_block_t(DecodeStateT<NH>& st, const uint32_t (&qb)[NH][8][2], uint8_t* stage,
                                                int valid, const float (&gb)[NH][2], float scale_log2, int slot,
-                                               int lane) {
+                                               int lane, bool outer = false) {
     using TG = TileGeom<64>;
     const int tok0 = slot * 16;
     if (tok0 >= valid) return;
@@ -307,8 +322,9 @@ __device__ __forceinline__ void decode_block_t(DecodeStateT<NH>& st, const uint3
     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-            s[nh][x] = v0 ? fmaf(s[nh][x], scale_log2, gb[nh][x]) : -INFINITY;
-            s[nh][2 + x] = v1 ? fmaf(s[nh][2 + x], scale_log2, gb[nh][x]) : -INFINITY;
+            const float bias = outer ? 0.f : gb[nh][x];
+            s[nh][x] = v0 ? fmaf(s[nh][x], scale_log2, bias) : -INFINITY;
+            s[nh][2 + x] = v1 ? fmaf(s[nh][2 + x], scale_log2, bias) : -INFINITY;
             float mx = fmaxf(s[nh][x], s[nh][2 + x]);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -340,6 +356,13 @@ __device__ __forceinline__ void decode_block_t(DecodeStateT<NH>& st, const uint3
         for (int e = 0; e < 4; ++e) p[e] = exp2f(s[nh][e] - u[nh][e & 1]);
         st.l[nh][0] += p[0] + p[2];
         st.l[nh][1] += p[1] + p[3];
+        if (outer) {  // the block's gate weights its values, not its share of the normaliser
+            const float gm0 = exp2f(gb[nh][0]), gm1 = exp2f(gb[nh][1]);
+            p[0] *= gm0;
+            p[2] *= gm0;
+            p[1] *= gm1;
+            p[3] *= gm1;
+        }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {  // tokens tr (hh = 0) and tr + 8 (hh = 1)
             const __nv_bfloat162 hi = __floats2bfloat162_rn(p[2 * hh], p[2 * hh + 1]);

@@ -7,9 +7,10 @@
 //  - one thread-block CLUSTER of C CTAs (one CTA per SM) per (sequence, KV
 //    group); CTA r owns slice r of the sequence's scored blocks and share r
 //    of the selected blocks for attention;
-//  - descriptors stream into a shared-memory ring as 16-byte cp.async gathers
-//    (one warp-wide instruction per 512-byte descriptor, completion tracked by
-//    the stage's mbarrier); K/V tiles with 2-D TMA loads (128-B swizzle);
+//  - one shared-memory ring of 32 KB stages, filled by a producer warp: a
+//    contiguous cache's descriptors arrive 64 per stage in one 4-D TMA load,
+//    a paged cache's are streamed by every warp with 16-byte loads straight
+//    into registers; K/V tiles come with 2-D TMA loads (128-B swizzle);
 //  - the selection is distributed: each CTA pushes the maxima of groups of its
 //    scores to its peers (distributed shared memory); every CTA derives the same
 //    lower bound T0 of the n-th score from them (k group maxima are k distinct
@@ -19,12 +20,14 @@
 //  - partial (O, LSE) of the CTAs are pushed to the merging CTA of each output
 //    element; all pushes precede a cluster barrier, after which every CTA reads
 //    only its own shared memory;
-//  - the appended tokens are written by CTA 0 before the first cluster barrier,
-//    and the descriptors of the touched blocks are recomputed from the K tiles
-//    the decode stages anyway (the touched blocks are local, hence selected).
-//    When a touched block is one the step itself scores (e.g. no local
-//    blocks), CTA 0 refreshes it from global memory first and a cluster barrier
-//    orders that before the scoring.
+//  - every CTA loads a 1/C share of the step's appended K/V rows at the start
+//    and stores it after scoring, ahead of the cluster barrier that precedes
+//    the decode's tile loads; the descriptors of the touched blocks are
+//    recomputed by the producer warp from the K tiles the decode stages anyway
+//    (the touched blocks are local, hence selected).  When a touched block is
+//    one the step itself scores (e.g. no local blocks), CTA 0 appends and
+//    refreshes it from global memory first and a cluster barrier orders that
+//    before the scoring.
 // No workspace: every intermediate lives in shared memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -631,7 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = f % NSt;
                 if (alive) alive = mbar_wait(&full[st], (f / NSt) & 1, c.status);
                 const int cb = j0 + (f - skip) * kSC;
-                const int nblk = f < skip ? 0 : min(kSC, js1 - cb);  // (<= 0: a drained fill)
+                // (<= 0: a drained fill, or a stage whose wait ran out: nothing of it is read)
+                const int nblk = (f < skip || !alive) ? 0 : min(kSC, js1 - cb);
                 const uint8_t* stage = dyn + (size_t)st * TG::kStage;
                 if (kScorer == SBA_SCORER_QUEST) {
 #pragma unroll
@@ -754,8 +758,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------- phase 2: distributed selection ----------------
     if (kScorer == SBA_SCORER_GATE) {
-        // per-head (max, sum exp(u - max)) over this CTA's scored blocks, pushed to every CTA
-        for (int g = warp; g < G; g += kThreads / 32) {
+        // softmax gates: per-head (max, sum exp(u - max)) over this CTA's scored blocks, pushed to
+        // every CTA; sigmoid and unnormalised gates need no normaliser (lse = 0 below)
+        const bool softmax_gate = a.p.gate_act == SBA_GATE_SOFTMAX;
+        for (int g = warp; softmax_gate && g < G; g += kThreads / 32) {
             float m = -INFINITY;
             for (int i = lane; i < js1 - j0; i += 32) m = fmaxf(m, u_s[g * ustride + i]);
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
@@ -773,8 +779,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 st_peer_f32(peer_addr(&mz_all[r * G + g][1], p), z);
             }
         }
-        cluster_sync();  // gate round: every CTA's softmax partials pushed
-        if (tid < G) {
+        if (softmax_gate) cluster_sync();  // gate round: every CTA's softmax partials pushed
+        if (tid < G && !softmax_gate) lse_s[tid] = 0.f;
+        if (tid < G && softmax_gate) {
             float M = -INFINITY;
             for (int p = 0; p < C; ++p) M = fmaxf(M, mz_all[p * G + tid][0]);
             float Z = 0.f;
@@ -786,17 +793,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             lse_s[tid] = M > -INFINITY ? M + logf(Z) : -INFINITY;
         }
         __syncthreads();
-        // group score of my ranked blocks: sum over the group of g = exp(u - LSE), four blocks per
-        // thread, pushed to every CTA
+        // group score of my ranked blocks: sum over the group of g (softmax: exp(u - LSE); raw:
+        // exp(u); sigmoid: 1 / (1 + exp(-u))), four blocks per thread, pushed to every CTA
+        const bool sigmoid_gate = a.p.gate_act == SBA_GATE_SIGMOID;
         for (int v = tid; 4 * v < jc1 - j0; v += kThreads) {
             const int jl = 4 * v;
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             for (int g = 0; g < G; ++g) {
                 const float4 u4 = *reinterpret_cast<const float4*>(u_s + g * ustride + jl);
-                sc[0] += expf(u4.x - lse_s[g]);
-                sc[1] += expf(u4.y - lse_s[g]);
-                sc[2] += expf(u4.z - lse_s[g]);
-                sc[3] += expf(u4.w - lse_s[g]);
+                if (sigmoid_gate) {
+                    sc[0] += gate_of(u4.x, 0.f, SBA_GATE_SIGMOID);
+                    sc[1] += gate_of(u4.y, 0.f, SBA_GATE_SIGMOID);
+                    sc[2] += gate_of(u4.z, 0.f, SBA_GATE_SIGMOID);
+                    sc[3] += gate_of(u4.w, 0.f, SBA_GATE_SIGMOID);
+                } else {
+                    sc[0] += expf(u4.x - lse_s[g]);
+                    sc[1] += expf(u4.y - lse_s[g]);
+                    sc[2] += expf(u4.z - lse_s[g]);
+                    sc[3] += expf(u4.w - lse_s[g]);
+                }
             }
             uint32_t kk[4];
 #pragma unroll
@@ -1096,8 +1111,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int fi = 0; fi < (i1 - i0) * kSub; ++fi, ++fill) {
             if ((int)(fill & 1) != grp) continue;  // the other group's fill
             const int st = fill % NSt;
-            if (alive) alive = mbar_wait(&full[st], (fill / NSt) & 1, c.status);
-            const StageInfo inf = info[st];
+            if (alive) {
+                alive = mbar_wait(&full[st], (fill / NSt) & 1, c.status);
+                // a wait that ran out leaves this warp's partial empty: after a timeout (reported
+                // in the status word) the merge sees no tokens from it rather than a stale stage
+                if (!alive) decode_state_init_t<kNH>(dst);
+            }
+            const StageInfo inf = alive ? info[st] : StageInfo{0, 0, 0, 0};
             uint8_t* stage = dyn + (size_t)st * TG::kStage;
             if (inf.ok) {
                 // SAS log-gate of this block (natural log) for this lane's heads, 0 for the current
@@ -1112,7 +1132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int x = 0; x < 2; ++x) {
                             const int hd = nh * 8 + 2 * t4 + x;
-                            if (hd < G) gb[nh][x] = ld_peer_f32(peer_addr(u_s + hd * ustride + off, owner)) - lse_s[hd];
+                            if (hd < G) gb[nh][x] = log_gate_of(ld_peer_f32(peer_addr(u_s + hd * ustride + off, owner)),
+                                                                lse_s[hd], a.p.gate_act);
                         }
                 }
                 if (kScorer == SBA_SCORER_GATE && a.gate_bias && gw == 0 && lane < 4 && inf.pos < a.n_max &&
@@ -1125,9 +1146,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (hd < G) a.gate_bias[((int64_t)s * c.H_q + h * G + hd) * a.n_max + inf.pos] = gb[nh][x];
                         }
                 }
+                // the gate in the attention: inside the softmax, on the values, or not at all
+                const float gsc = (kScorer == SBA_SCORER_GATE && a.p.log_gate != SBA_LOG_GATE_OFF) ? kLog2e : 0.f;
 #pragma unroll
-                for (int nh = 0; nh < kNH; ++nh) gb[nh][0] *= kLog2e, gb[nh][1] *= kLog2e;
-                if (alive) decode_block_t<kNH>(dst, qb, stage, inf.valid, gb, a.scale_log2, gw, lane);
+                for (int nh = 0; nh < kNH; ++nh) gb[nh][0] *= gsc, gb[nh][1] *= gsc;
+                decode_block_t<kNH>(dst, qb, stage, inf.valid, gb, a.scale_log2, gw, lane,
+                                    kScorer == SBA_SCORER_GATE && a.p.log_gate == SBA_LOG_GATE_OUTER);
             }
             fence_proxy_async_smem();
             __syncwarp();

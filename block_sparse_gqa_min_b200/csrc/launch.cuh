@@ -65,6 +65,10 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStr
     return SBA_OK;
 }
 
+// Host-side argument checks of sba_score_select, short of the workspace (api.cu).
+int check_score_select(const sba_cache* c, const void* q, const sba_select_params* p, const int32_t* sel_idx,
+                       const int32_t* sel_cnt, int32_t n_max);
+
 // Host-side entry points of the kernel files (validated arguments only).
 int launch_append_kv(const sba_cache& c, const void* k_new, const void* v_new, const int32_t* pos_start, int n_new,
                      cudaStream_t stream);
@@ -72,16 +76,20 @@ int launch_update_descriptors(const sba_cache& c, const int32_t* pos_start, int 
                               cudaStream_t stream);
 int score_chunk_blocks(const sba_cache& c);
 size_t score_workspace_bytes(const sba_cache& c, const sba_select_params& p);
-int launch_score_select(const sba_cache& c, const void* q, const sba_select_params& p, int32_t* sel_idx,
+int launch_score_select(const sba_cache& c, const void* q, int M, const sba_select_params& p, int32_t* sel_idx,
                         int32_t* sel_cnt, float* gate_bias, int n_max, void* ws, cudaStream_t stream);
 int launch_sparse_decode(const sba_cache& c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
                          const float* gate_bias, int n_max, float scale, int num_splits, float* o_part,
-                         float* lse_part, cudaStream_t stream);
+                         float* lse_part, bool outer, cudaStream_t stream);
 int step_cluster_size(const sba_cache& c, const sba_select_params& p, int num_sms);
 int launch_decode_step(const sba_cache& c, const void* q, const void* k_new, const void* v_new,
                        const int32_t* pos_start, int n_new, const float* gate_A, const sba_select_params& p,
                        float scale, void* out, int out_dtype, float* lse_out, int32_t* sel_idx, int32_t* sel_cnt,
                        float* gate_bias, int n_max, int cluster, cudaStream_t stream);
+int mq_row_groups(const sba_cache& c, int M);
+int launch_multi_query(const sba_cache& c, const void* q, int M, const int32_t* sel_idx, const int32_t* sel_cnt,
+                       int n_max, const void* k_new, const void* v_new, bool dense, float scale, int num_splits,
+                       float* o_part, float* lse_part, cudaStream_t stream);
 int launch_fold_gate(const float* Wq, const float* Wk, int dg, float* A, cudaStream_t stream);
 int launch_combine(const float* o_part, const float* lse_part, int B, int H_q, int S, void* out, int out_dtype,
                    float* lse_out, cudaStream_t stream);

@@ -5,8 +5,9 @@
 // heads of a GQA group share one selection; Key points: top-n that always
 // keeps the recent local blocks and a minimum count.
 // "SAS: Simple Attention Sparsification ...", Method: gate scores are
-// softmax-normalised over the historical blocks; the current block B0 keeps a
-// unit gate; the log-gates of the selected blocks go into the attention logits.
+// softmax-normalised over the historical blocks (or, as in its ablations,
+// passed through a sigmoid or injected unnormalised); the current block B0
+// keeps a unit gate; the log-gates of the selected blocks go into the attention.
 //
 // One launch per call.  CTAs of grid (chunk, kv head, sequence) score CHUNK
 // blocks each and write fp32 scores to the workspace; the last CTA to finish a
@@ -37,7 +38,8 @@ constexpr int kSelCap = 1024;  // selection buffer (candidates above the group-m
 
 struct ScoreArgs {
     sba_cache c;
-    const __nv_bfloat16* q;
+    const __nv_bfloat16* q;  // [B][M][H_q][d]
+    int M;                   // query tokens per sequence sharing the selection (Quest)
     sba_select_params p;
     int32_t* sel_idx;
     int32_t* sel_cnt;
@@ -121,8 +123,11 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
         float coef[64];
 #pragma unroll
         for (int e = 0; e < 64; ++e) coef[e] = 0.f;
-        for (int g = 0; g < G; ++g) {
-            const uint4* qp = reinterpret_cast<const uint4*>(a.q + ((int64_t)s * c.H_q + h * G + g) * kHeadDim + ch0);
+        // (several query tokens of a sequence: their heads join the group's sum, ReSA Summary)
+        for (int gi = 0; gi < G * a.M; ++gi) {
+            const int g = gi % G, qi = gi / G;
+            const uint4* qp = reinterpret_cast<const uint4*>(
+                a.q + (((int64_t)s * a.M + qi) * c.H_q + h * G + g) * kHeadDim + ch0);
 #pragma unroll
             for (int k8 = 0; k8 < 8; ++k8) {
                 const uint4 w = __ldg(qp + k8);
@@ -251,7 +256,10 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
         for (int j = tid; j < NC; j += kThreads) keys[j] = orderable_key(__ldcg(sc + j));
     } else {
         const int n_chunks = gridDim.x;
-        for (int g = warp; g < G; g += kWarps) {
+        const int act = a.p.gate_act;  // sigmoid and unnormalised gates need no normaliser
+        if (act != SBA_GATE_SOFTMAX)
+            for (int g = tid; g < G; g += kThreads) lse_s[g] = 0.f;
+        for (int g = warp; act == SBA_GATE_SOFTMAX && g < G; g += kWarps) {
             const float* mzp = a.mz + ((int64_t)s * c.H_q + h * G + g) * n_chunks * 2;
             float M = -INFINITY;
             for (int i = lane; i < n_chunks; i += 32) M = fmaxf(M, __ldcg(mzp + 2 * i));
@@ -271,7 +279,7 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
         for (int j = tid; j < NC; j += kThreads) {
             float sc = 0.f;
             for (int g = 0; g < G; ++g)
-                sc += expf(__ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j) - lse_s[g]);
+                sc += gate_of(__ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j), lse_s[g], act);
             keys[j] = orderable_key(sc);
         }
     }
@@ -293,8 +301,9 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
         for (int i = tid; i < n_out * G; i += kThreads) {
             const int pos = i / G, g = i % G;
             const int j = __ldcg(out + pos);
-            const float bias =
-                j == N - 1 ? 0.f : __ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j) - lse_s[g];
+            const float bias = j == N - 1 ? 0.f
+                                          : log_gate_of(__ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j),
+                                                        lse_s[g], a.p.gate_act);
             a.gate_bias[((int64_t)s * c.H_q + h * G + g) * a.n_max + pos] = bias;
         }
     }
@@ -321,13 +330,14 @@ static size_t score_smem_bytes(const sba_cache& c, int chunk) {
     return (main_words + chunk + sel_words) * 4;
 }
 
-int launch_score_select(const sba_cache& c, const void* q, const sba_select_params& p, int32_t* sel_idx,
+int launch_score_select(const sba_cache& c, const void* q, int M, const sba_select_params& p, int32_t* sel_idx,
                         int32_t* sel_cnt, float* gate_bias, int n_max, void* ws, cudaStream_t stream) {
     const int chunk = score_chunk_blocks(c);
     const WsLayout w = ws_layout(c, p, chunk);
     ScoreArgs a{};
     a.c = c;
     a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.M = M;
     a.p = p;
     a.sel_idx = sel_idx;
     a.sel_cnt = sel_cnt;

@@ -32,6 +32,13 @@ SBA_SCORER_GATE = 1
 SBA_OUT_F32 = 0
 SBA_OUT_BF16 = 1
 
+SBA_LOG_GATE_OFF = 0
+SBA_LOG_GATE_INNER = 1
+SBA_LOG_GATE_OUTER = 2
+SBA_GATE_SOFTMAX = 0
+SBA_GATE_SIGMOID = 1
+SBA_GATE_RAW = 2
+
 
 class SbaError(RuntimeError):
     def __init__(self, code: int, where: str):
@@ -74,6 +81,8 @@ class sba_select_params(ctypes.Structure):
         ("keep_num", ctypes.c_int32),
         ("keep_den", ctypes.c_int32),
         ("scorer", ctypes.c_int32),
+        ("log_gate", ctypes.c_int32),
+        ("gate_act", ctypes.c_int32),
     ]
 
 
@@ -92,6 +101,14 @@ _SIGS = {
                           ctypes.c_size_t, _P], ctypes.c_int),
     "sba_sparse_decode": ([ctypes.POINTER(sba_cache), _P, _P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _P],
                           ctypes.c_int),
+    "sba_sparse_decode_outer": ([ctypes.POINTER(sba_cache), _P, _P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _P],
+                                ctypes.c_int),
+    "sba_score_select_multi": ([ctypes.POINTER(sba_cache), _P, _I, ctypes.POINTER(sba_select_params), _P, _P, _I,
+                                _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "sba_sparse_decode_multi": ([ctypes.POINTER(sba_cache), _P, _I, _P, _P, _I, ctypes.c_float, _I, _P, _P, _P],
+                                ctypes.c_int),
+    "sba_multi_row_groups": ([ctypes.POINTER(sba_cache), _I], _I),
+    "sba_rectify": ([ctypes.POINTER(sba_cache), _P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _P], ctypes.c_int),
     "sba_combine": ([_P, _P, _I, _I, _I, _I, _P, _I, _P, _P], ctypes.c_int),
     "sba_fold_gate": ([ctypes.POINTER(sba_gate), _P, _P], ctypes.c_int),
     "sba_static_scratch_bytes": ([], ctypes.c_size_t),
@@ -193,8 +210,9 @@ class Cache:
         return cached[1]
 
 
-def select_params(n_budget=0, n_local=0, n_min=0, keep_num=0, keep_den=0, scorer=SBA_SCORER_QUEST):
-    return sba_select_params(n_budget, n_local, n_min, keep_num, keep_den, scorer)
+def select_params(n_budget=0, n_local=0, n_min=0, keep_num=0, keep_den=0, scorer=SBA_SCORER_QUEST,
+                  log_gate=SBA_LOG_GATE_OFF, gate_act=SBA_GATE_SOFTMAX):
+    return sba_select_params(n_budget, n_local, n_min, keep_num, keep_den, scorer, log_gate, gate_act)
 
 
 def sba_status_string(code: int) -> str:
@@ -266,8 +284,54 @@ def sba_sparse_decode(c: Cache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt:
                                     _ptr(lse_part), _stream(stream)), "sba_sparse_decode")
 
 
+def sba_sparse_decode_outer(c: Cache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
+                            gate_bias: torch.Tensor, softmax_scale: float, o_part: torch.Tensor,
+                            lse_part: torch.Tensor, stream=None):
+    n_max = int(sel_idx.shape[-1])
+    num_splits = int(lse_part.shape[-1])
+    _check(load().sba_sparse_decode_outer(ctypes.byref(c.struct()), _ptr(q), _ptr(sel_idx), _ptr(sel_cnt),
+                                          _ptr(gate_bias), n_max, float(softmax_scale), num_splits, _ptr(o_part),
+                                          _ptr(lse_part), _stream(stream)), "sba_sparse_decode_outer")
+
+
+def sba_score_select_multi(c: Cache, q: torch.Tensor, p: sba_select_params, sel_idx: torch.Tensor,
+                           sel_cnt: torch.Tensor, ws: torch.Tensor, stream=None):
+    """q: bf16 [B][M][H_q][d]; one Quest selection per (sequence, group) for all M tokens."""
+    M = int(q.shape[1])
+    n_max = int(sel_idx.shape[-1])
+    _check(load().sba_score_select_multi(ctypes.byref(c.struct()), _ptr(q), M, ctypes.byref(p), _ptr(sel_idx),
+                                         _ptr(sel_cnt), n_max, _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "sba_score_select_multi")
+
+
+def sba_multi_row_groups(c: Cache, M: int) -> int:
+    return int(load().sba_multi_row_groups(ctypes.byref(c.struct()), M))
+
+
+def sba_sparse_decode_multi(c: Cache, q: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
+                            softmax_scale: float, o_part: torch.Tensor, lse_part: torch.Tensor, stream=None):
+    """q: bf16 [B][M][H_q][d]; o_part fp32 [B][M][H_q][S][d], lse_part [B][M][H_q][S]."""
+    M = int(q.shape[1])
+    n_max = int(sel_idx.shape[-1])
+    num_splits = int(lse_part.shape[-1])
+    _check(load().sba_sparse_decode_multi(ctypes.byref(c.struct()), _ptr(q), M, _ptr(sel_idx), _ptr(sel_cnt), n_max,
+                                          float(softmax_scale), num_splits, _ptr(o_part), _ptr(lse_part),
+                                          _stream(stream)), "sba_sparse_decode_multi")
+
+
+def sba_rectify(c: Cache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, softmax_scale: float,
+                o_part: torch.Tensor, lse_part: torch.Tensor, stream=None):
+    """q: bf16 [B][f][H_q][d]; k_new, v_new bf16 [B][f][H_kv][d] (the last f positions)."""
+    f = int(q.shape[1])
+    num_splits = int(lse_part.shape[-1])
+    _check(load().sba_rectify(ctypes.byref(c.struct()), _ptr(q), _ptr(k_new), _ptr(v_new), f, float(softmax_scale),
+                              num_splits, _ptr(o_part), _ptr(lse_part), _stream(stream)), "sba_rectify")
+
+
 def sba_combine(o_part: torch.Tensor, lse_part: torch.Tensor, out: torch.Tensor,
                 lse_out: Optional[torch.Tensor] = None, stream=None):
+    if o_part.dim() == 5:  # multi-token partials [B][M][H_q][S][d]: merge M*H_q rows
+        o_part = o_part.view(o_part.shape[0], -1, o_part.shape[3], o_part.shape[4])
     B, H_q, S, d = o_part.shape
     dt = SBA_OUT_BF16 if out.dtype == torch.bfloat16 else SBA_OUT_F32
     if out.dtype not in (torch.bfloat16, torch.float32):
@@ -341,8 +405,14 @@ def alloc_step(c: Cache, p: sba_select_params, num_splits: Optional[int] = None,
 
 def decode_step(c: Cache, q: torch.Tensor, p: sba_select_params, bufs: StepBuffers, softmax_scale: float,
                 stream=None):
-    """score_select -> sparse_decode -> combine for one layer (three library calls)."""
+    """score_select -> sparse_decode -> combine for one layer (three library calls; the gate's
+    position p.log_gate picks the decode call and whether it gets the log-gates)."""
     sba_score_select(c, q, p, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, bufs.ws, stream)
-    sba_sparse_decode(c, q, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, softmax_scale, bufs.o_part, bufs.lse_part,
-                      stream)
+    gate = p.scorer == SBA_SCORER_GATE
+    if gate and p.log_gate == SBA_LOG_GATE_OUTER:
+        sba_sparse_decode_outer(c, q, bufs.sel_idx, bufs.sel_cnt, bufs.gate_bias, softmax_scale, bufs.o_part,
+                                bufs.lse_part, stream)
+    else:
+        bias = bufs.gate_bias if (gate and p.log_gate == SBA_LOG_GATE_INNER) else None
+        sba_sparse_decode(c, q, bufs.sel_idx, bufs.sel_cnt, bias, softmax_scale, bufs.o_part, bufs.lse_part, stream)
     sba_combine(bufs.o_part, bufs.lse_part, bufs.out, bufs.lse, stream)

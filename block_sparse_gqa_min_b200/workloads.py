@@ -16,8 +16,9 @@ Workloads (one decode step of every layer):
                   per (layer, kv head, channel); Quest scorer.
   r1_7b_256k      28 layers x 28 Q / 4 KV heads (GQA 7), len 262144, b 128,
                   sparsity p = 0.95 (keep 5/100 of the blocks, rounded up),
-                  4 local, min 16; N(0,1); Quest; a 32-token rectification
-                  window re-appended (f = 32).
+                  4 local, min 16; N(0,1); Quest; one token appended per
+                  step and, every f = 32 steps, the rectification pass of the
+                  last 32 tokens (their queries, keys and values ~ N(0,1)).
   paged_b8        batch 8, 36 layers x 32/8 heads, lengths ~ U[32768, 65536],
                   64-token pages at a seed-shuffled permutation of physical
                   slots through a block table, budget 32 blocks (2048 tokens),
@@ -59,6 +60,9 @@ class Workload:
     channel_scale_sigma: float = 0.0
     append_tokens: int = 1      # tokens re-appended per step (rectification window)
     dg: int = 128               # gate width
+    gate_position: str = "inner"  # gate scorer: "inner" (log g in the logits), "outer" (g on V), "off"
+    gate_act: str = "softmax"     # gate scorer: "softmax", "sigmoid" or "raw"
+    rectify_every: int = 0        # f: a dense rectification pass of the last f tokens every f steps
 
     @property
     def G(self) -> int:
@@ -87,7 +91,7 @@ WORKLOADS = {
                          len_hi=32768, n_budget=64, n_local=2, n_min=16, channel_scale_sigma=0.5),
     "r1_7b_256k": Workload("r1_7b_256k", B=1, H_q=28, H_kv=4, d=128, b=128, layers=28,
                            len_lo=262144, len_hi=262144, n_local=4, n_min=16, keep_num=5,
-                           keep_den=100, append_tokens=32),
+                           keep_den=100, rectify_every=32),
     "paged_b8": Workload("paged_b8", B=8, H_q=32, H_kv=8, d=128, b=64, layers=36, len_lo=32768,
                          len_hi=65536, n_budget=32, n_local=2, n_min=16, paged=True),
     "qwen3_14b_gate": Workload("qwen3_14b_gate", B=1, H_q=40, H_kv=8, d=128, b=64, layers=40,
@@ -199,6 +203,25 @@ def make_layer(w: Workload, lay: Layout, seed: int, layer: int, device="cpu") ->
         out.Wq = torch.randn((w.dg, w.d), generator=g, device=dev, dtype=torch.float32) / math.sqrt(w.d)
         out.Wk = torch.randn((w.dg, 3 * w.d), generator=g, device=dev, dtype=torch.float32) / math.sqrt(3 * w.d)
     return out
+
+
+@dataclass
+class RectInputs:
+    q: torch.Tensor                 # bf16 [B][f][H_q][d]: the window's query tokens
+    k_new: torch.Tensor             # bf16 [B][f][H_kv][d]: their re-encoded keys and values
+    v_new: torch.Tensor
+
+
+def make_rect_inputs(w: Workload, seed: int, layer: int, device="cpu") -> RectInputs:
+    """Synthetic inputs of one layer's rectification pass (f = w.rectify_every tokens),
+    all ~ N(0,1) in bf16 from their own seeded generator."""
+    f = w.rectify_every
+    dev = torch.device(device)
+    g = make_generator(dev, seed * 1_000_033 + layer * 103 + 7)
+    q = torch.randn((w.B, f, w.H_q, w.d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    kn = torch.randn((w.B, f, w.H_kv, w.d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vn = torch.randn((w.B, f, w.H_kv, w.d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    return RectInputs(q, kn, vn)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

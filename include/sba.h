@@ -33,6 +33,10 @@
  *    rejected on the host (nothing is enqueued then) or a launch fails.
  *    Faults of already-enqueued kernels surface at the caller's next
  *    synchronisation, as usual for CUDA.  No C++ exception crosses the ABI.
+ *  - The library remembers, per device, the kernel attributes it has set
+ *    (shared-memory limits, cluster sizes).  A cudaDeviceReset discards them
+ *    on the device; a process that resets a device reloads the library before
+ *    using it there again (calls otherwise fail with SBA_ERR_CUDA).
  *  - Data-dependent problems found on the device (a block-table entry outside
  *    [0, num_pages), a position outside the table, a selected index outside
  *    [0, N), a wait that timed out) never trap: the offending access is
@@ -72,6 +76,18 @@ extern "C" {
 
 #define SBA_OUT_F32 0
 #define SBA_OUT_BF16 1
+
+/* Where the gate enters the attention ("SAS ...", Method: the gate may sit
+ * inside the softmax or outside it, on the values). */
+#define SBA_LOG_GATE_OFF 0    /* the gates select blocks only: o = softmax(l) V */
+#define SBA_LOG_GATE_INNER 1  /* o = softmax(l + log g) V (log g per selected block) */
+#define SBA_LOG_GATE_OUTER 2  /* o = softmax(l) (g . V): each token's value times its block's gate */
+
+/* Gate activation phi, g = phi(u) on the historical blocks ("SAS ...", Method
+ * and its ablations: softmax, sigmoid and unnormalised logit injection). */
+#define SBA_GATE_SOFTMAX 0  /* g = softmax of u over the C = N-1 historical blocks */
+#define SBA_GATE_SIGMOID 1  /* g = 1 / (1 + exp(-u)), each block on its own */
+#define SBA_GATE_RAW 2      /* unnormalised: log g = u (g = exp(u)) */
 
 /* The KV cache of ONE attention layer, and its block descriptors.
  *
@@ -124,14 +140,24 @@ typedef struct sba_gate {
  * {N-L .. N-1} are always kept and the rest are the top scores of blocks
  * 0 .. N-L-1 (fp32 score descending, then index ascending; -0 == +0).
  * With the gate scorer the current block B0 = N-1 is always kept, i.e. L >= 1
- * ("SAS ...", Method). */
+ * ("SAS ...", Method).
+ * Gate scorer only (ignored by Quest, where they must be 0):
+ *  - gate_act: phi of the gates g = phi(u) (SBA_GATE_*).  The group ranks the
+ *    historical blocks by sum over its heads of g; the log-gate of a selected
+ *    historical block is log g, and 0 for B0 (unit gate).  With
+ *    SBA_GATE_RAW, exp(u) must stay finite in fp32 (u < 88).
+ *  - log_gate: whether and where the gate enters the attention of
+ *    sba_decode_step (SBA_LOG_GATE_*).  The split-KV calls take the choice
+ *    through which decode call is made (see sba_sparse_decode). */
 typedef struct sba_select_params {
     int32_t n_budget;
     int32_t n_local;
     int32_t n_min;
     int32_t keep_num;
     int32_t keep_den;
-    int32_t scorer; /* SBA_SCORER_QUEST or SBA_SCORER_GATE */
+    int32_t scorer;   /* SBA_SCORER_QUEST or SBA_SCORER_GATE */
+    int32_t log_gate; /* SBA_LOG_GATE_OFF, _INNER or _OUTER */
+    int32_t gate_act; /* SBA_GATE_SOFTMAX, _SIGMOID or _RAW */
 } sba_select_params;
 
 /* Message for a status code (static string, never NULL). */
@@ -187,9 +213,10 @@ int sba_update_descriptors(const sba_cache *c, const int32_t *pos_start, int32_t
  *    sum_c max(q_qh,c * min_jc, q_qh,c * max_jc), an upper bound of
  *    max_t q.k_t over the block, in fp32.
  *  - Gate ("SAS ...", Method): u_qh,j = q_qh . kg_j over the historical blocks
- *    j < N-1, g = softmax_j(u), score = sum over the group of g.  When
- *    gate_bias != NULL it receives log g_qh,j = u_qh,j - logsumexp_j(u_qh) for
- *    every selected historical block and 0 for B0 = N-1.
+ *    j < N-1, g = phi(u) with phi = p->gate_act (softmax over j by default),
+ *    score = sum over the group of g.  When gate_bias != NULL it receives
+ *    log g_qh,j (softmax: u_qh,j - logsumexp_j(u_qh); sigmoid: log sigmoid(u);
+ *    raw: u) for every selected historical block and 0 for B0 = N-1.
  * q          device bf16 [B][H_q][d].
  * sel_idx    device int32 [B][H_kv][n_max]: selected logical block indices,
  *            ascending; entries past sel_cnt are left unchanged.
@@ -221,6 +248,17 @@ int sba_sparse_decode(const sba_cache *c, const void *q, const int32_t *sel_idx,
                       float softmax_scale, int32_t num_splits, float *o_part, float *lse_part,
                       void *stream);
 
+/* sba_sparse_decode with the gate OUTSIDE the softmax ("SAS ...", Method: the
+ * gate may scale the values instead of entering the logits).  Same arguments;
+ * gate_bias (log g, as sba_score_select writes it) is required.  Per split:
+ *   o_part = sum_t softmax(l)_t g_j(t) v_t,  l_t = (q . k_t) * softmax_scale,
+ *   lse_part = log sum_t exp(l_t)  (the ungated logits),
+ * so sba_combine of the splits gives o = softmax(q K^T * scale) (g . V). */
+int sba_sparse_decode_outer(const sba_cache *c, const void *q, const int32_t *sel_idx,
+                            const int32_t *sel_cnt, const float *gate_bias, int32_t n_max,
+                            float softmax_scale, int32_t num_splits, float *o_part,
+                            float *lse_part, void *stream);
+
 /* Log-sum-exp merge of the splits (Flash-Decoding, cited by "Rectified Sparse
  * Attention ...", References): out = sum_s w_s o_s with
  * w_s = exp(lse_s - LSE), LSE = log sum_s exp(lse_s).  All splits -inf gives
@@ -231,6 +269,54 @@ int sba_sparse_decode(const sba_cache *c, const void *q, const int32_t *sel_idx,
 int sba_combine(const float *o_part, const float *lse_part, int32_t B, int32_t H_q,
                 int32_t num_splits, int32_t d, void *out, int32_t out_dtype, float *lse_out,
                 void *stream);
+
+/* Several query tokens per sequence sharing one selection ("Rectified Sparse
+ * Attention ...", Summary: the f tokens re-encoded together, every query head
+ * of a GQA group sharing one block selection; Key points: the comparison with
+ * self-speculative decoding, which checks several draft tokens at once).
+ * The M query tokens of sequence s sit at its last M positions, len_s-M ..
+ * len_s-1 (their keys and values already in the cache), and token i attends
+ * causally to positions t <= len_s-M+i.  Quest scorer only.
+ *
+ * sba_score_select_multi: as sba_score_select, with the Quest score of a block
+ * summed over the group's G heads AND the M tokens (the M*G query rows act as
+ * one group); one selection per (sequence, KV group).
+ * q  device bf16 [B][M][H_q][d].  Other arguments as sba_score_select. */
+int sba_score_select_multi(const sba_cache *c, const void *q, int32_t M, const sba_select_params *p,
+                           int32_t *sel_idx, int32_t *sel_cnt, int32_t n_max, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* sba_sparse_decode for M query tokens: every query row (token i, head qh)
+ * attends over the group's selected blocks, masked causally (t <= len-M+i) and
+ * at len.  Writes o_part fp32 [B][M][H_q][S][d] and lse_part [B][M][H_q][S]
+ * (-inf for a row that saw no token), so sba_combine with H_q' = M*H_q merges
+ * the splits into [B][M][H_q][d].  The M*G rows of a group run in row groups
+ * of 128 (sba_multi_row_groups), each a CTA per split: choose num_splits so
+ * that B*H_kv*row_groups*num_splits fills the GPU. */
+int sba_sparse_decode_multi(const sba_cache *c, const void *q, int32_t M, const int32_t *sel_idx,
+                            const int32_t *sel_cnt, int32_t n_max, float softmax_scale,
+                            int32_t num_splits, float *o_part, float *lse_part, void *stream);
+
+/* Row groups (CTAs per split and KV head) of the multi-token calls: ceil(M*G/128). */
+int32_t sba_multi_row_groups(const sba_cache *c, int32_t M);
+
+/* The rectification pass ("Rectified Sparse Attention ...", Summary: every f
+ * generated tokens are re-encoded in one parallel dense pass that rewrites
+ * their KV entries, which bounds the error the sparse steps accumulate; Key
+ * points: f in {16, 32, 64, 128}).  The caller has already advanced seq_lens
+ * to include the f tokens, which sit at positions len_s-f .. len_s-1.  One
+ * launch:
+ *  1. writes k_new, v_new (device bf16 [B][f][H_kv][d]) at those positions
+ *     through the block table, overwriting what the sparse steps stored;
+ *  2. recomputes the Quest descriptors (c->desc, when non-NULL) of the blocks
+ *     those positions touch, from all of each block's valid keys;
+ *  3. dense causal attention of the f query tokens (q [B][f][H_q][d]) over
+ *     every block [0, N): outputs as sba_sparse_decode_multi with M = f.
+ * 1 <= f <= 128 and f <= len_s (a shorter sequence reports
+ * SBA_DEV_BAD_POSITION).  Gate keys are not refreshed here (call
+ * sba_update_descriptors for them). */
+int sba_rectify(const sba_cache *c, const void *q, const void *k_new, const void *v_new, int32_t f,
+                float softmax_scale, int32_t num_splits, float *o_part, float *lse_part, void *stream);
 
 /* Size in bytes of the static scratch behind sba_score_select_static (8 MiB). */
 size_t sba_static_scratch_bytes(void);
@@ -246,8 +332,9 @@ size_t sba_static_scratch_bytes(void);
  * loads it, until the process exits.
  *  - A problem needing more scratch than that (sba_workspace_size) returns
  *    SBA_ERR_WORKSPACE before anything is enqueued.
- *  - The first call on a device looks the array's address up for that device;
- *    make it before any stream capture.
+ *  - The first call on a device looks the array's address up for that device
+ *    (and again when the device's context has changed, e.g. after
+ *    cudaDeviceReset); make it before any stream capture.
  *  - All calls on a device share the array and it keeps the last call's
  *    contents; each call first clears the completion counters on `stream`
  *    (cudaMemsetAsync).  Calls whose kernels can overlap on the GPU (streams
@@ -279,7 +366,10 @@ int32_t sba_decode_step_cluster(const sba_cache *c, const sba_select_params *p);
  * 3-4. score and select exactly as sba_score_select;
  * 5-6. attention over the selected blocks and the merge, as sba_sparse_decode
  *    followed by sba_combine, writing out [B][H_q][d] (SBA_OUT_F32 or
- *    SBA_OUT_BF16) and lse_out [B][H_q] (fp32, may be NULL).
+ *    SBA_OUT_BF16) and lse_out [B][H_q] (fp32, may be NULL).  With the gate
+ *    scorer, p->log_gate places the gate: off (selection only), inside the
+ *    softmax (as sba_sparse_decode with gate_bias) or on the values (as
+ *    sba_sparse_decode_outer).
  * sel_idx/sel_cnt/gate_bias (layouts of sba_score_select, each may be NULL)
  * report the selection; n_max is their row length.
  * The caller advances seq_lens to include the appended tokens BEFORE the call.

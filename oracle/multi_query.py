@@ -41,10 +41,12 @@ def _truncated(c: Cache, seq_lens: np.ndarray) -> Cache:
 
 
 def decode_multi(c: Cache, q: np.ndarray, *, scale: float, n_budget: int, n_local: int, n_min: int,
-                 keep_num: int = 0, keep_den: int = 0, dense: bool = False, n_max: Optional[int] = None):
+                 keep_num: int = 0, keep_den: int = 0, dense: bool = False, n_max: Optional[int] = None,
+                 sel=None):
     """q: bf16 bits [B][M][H_q][d].  Returns (score [B][H_kv][max_blocks], sel_idx, sel_cnt,
     out [B][M][H_q][d], lse [B][M][H_q]); dense=True selects every block (the
-    rectification pass)."""
+    rectification pass); sel = (sel_idx, sel_cnt) replaces the top-n selection by a
+    given one (used to re-run a near-tie case)."""
     q = np.asarray(q, dtype=np.uint16)
     B, M = q.shape[0], q.shape[1]
     score = np.zeros((c.B, c.H_kv, c.max_blocks))
@@ -59,6 +61,8 @@ def decode_multi(c: Cache, q: np.ndarray, *, scale: float, n_budget: int, n_loca
         for s in range(c.B):
             sel_idx[s, :, : N[s]] = np.arange(N[s], dtype=np.int32)
             sel_cnt[s, :] = N[s]
+    elif sel is not None:
+        sel_idx, sel_cnt = (np.asarray(x, dtype=np.int32) for x in sel)
     else:
         sel_idx, sel_cnt = select(score, c.seq_lens, c.b, n_budget, n_local, n_min, keep_num, keep_den, n_max)
     out = np.zeros((B, M, c.H_q, c.d))

@@ -78,10 +78,12 @@ def log_gates(u: np.ndarray, activation: str) -> np.ndarray:
 
 def decode_variant(c: Cache, q: np.ndarray, Wq: np.ndarray, Wk: np.ndarray, *, scale: float, n_budget: int,
                    n_local: int, n_min: int, activation: str = "softmax", position: str = "inner",
-                   n_max: Optional[int] = None) -> Decoded:
+                   n_max: Optional[int] = None, sel=None) -> Decoded:
     """One decode step with a SAS gate variant: gates, group scores, selection
     (current block always kept), attention with the gate inside or outside the
-    softmax.  Returns the main oracle's Decoded record (logg = log g, 0 on B0)."""
+    softmax.  Returns the main oracle's Decoded record (logg = log g, 0 on B0).
+    sel = (sel_idx, sel_cnt) replaces the top-n selection by a given one (the
+    attention is then over those blocks; used to re-run a near-tie case)."""
     if position not in POSITIONS:
         raise ValueError(position)
     q = np.asarray(q, dtype=np.uint16)
@@ -101,7 +103,10 @@ def decode_variant(c: Cache, q: np.ndarray, Wq: np.ndarray, Wk: np.ndarray, *, s
             score[s, qh // c.G, : Ns - 1] += np.exp(lg)
     if n_max is None:
         n_max = max(1, c.max_blocks)
-    sel_idx, sel_cnt = select(score, c.seq_lens, c.b, n_budget, max(n_local, 1), n_min, n_max=n_max)
+    if sel is None:
+        sel_idx, sel_cnt = select(score, c.seq_lens, c.b, n_budget, max(n_local, 1), n_min, n_max=n_max)
+    else:
+        sel_idx, sel_cnt = (np.asarray(x, dtype=np.int32) for x in sel)
 
     qf = _bf16_to_f64(q)
     out = np.zeros((c.B, c.H_q, c.d))

@@ -83,16 +83,39 @@ def fill_descriptors(c, w: W.Workload, li: W.LayerInputs):
 def params_of(w: W.Workload):
     from block_sparse_gqa_min_b200 import sba
 
+    gate = w.scorer == "gate"
+    pos = {"off": sba.SBA_LOG_GATE_OFF, "inner": sba.SBA_LOG_GATE_INNER, "outer": sba.SBA_LOG_GATE_OUTER}
+    act = {"softmax": sba.SBA_GATE_SOFTMAX, "sigmoid": sba.SBA_GATE_SIGMOID, "raw": sba.SBA_GATE_RAW}
     return sba.select_params(w.n_budget, w.n_local, w.n_min, w.keep_num, w.keep_den,
-                             sba.SBA_SCORER_GATE if w.scorer == "gate" else sba.SBA_SCORER_QUEST)
+                             sba.SBA_SCORER_GATE if gate else sba.SBA_SCORER_QUEST,
+                             pos[w.gate_position] if gate else 0, act[w.gate_act] if gate else 0)
 
 
-def oracle_decode(w: W.Workload, oc: O.Cache, li: W.LayerInputs, n_max=None):
+def oracle_decode(w: W.Workload, oc: O.Cache, li: W.LayerInputs, n_max=None, sel=None):
+    """The oracle's whole step for workload w (the gate variants through
+    oracle.sas_variants); sel = (sel_idx, sel_cnt) re-runs it on a given selection."""
+    if w.scorer == "gate" and (w.gate_act != "softmax" or w.gate_position == "outer"):
+        from oracle import sas_variants as V
+
+        d = V.decode_variant(oc, W.bf16_bits(li.q), li.Wq.cpu().numpy(), li.Wk.cpu().numpy(), scale=w.scale,
+                             n_budget=w.n_budget, n_local=w.n_local, n_min=w.n_min, activation=w.gate_act,
+                             position=w.gate_position if w.gate_position != "off" else "inner", n_max=n_max,
+                             sel=sel)
+        if w.gate_position == "off":  # the gates select; the attention is plain
+            o, l = O.attend(oc, W.bf16_bits(li.q), d.sel_idx, d.sel_cnt, w.scale, None)
+            d = O.Decoded(d.score, d.sel_idx, d.sel_cnt, d.logg, o, l)
+        return d
     kw = dict(scale=w.scale, n_budget=w.n_budget, n_local=w.n_local, n_min=w.n_min,
-              keep_num=w.keep_num, keep_den=w.keep_den, scorer=w.scorer, n_max=n_max)
+              keep_num=w.keep_num, keep_den=w.keep_den, scorer=w.scorer, n_max=n_max,
+              log_gate=w.gate_position != "off")
     if w.scorer == "gate":
         kw.update(Wq=li.Wq.cpu().numpy(), Wk=li.Wk.cpu().numpy())
-    return O.decode(oc, W.bf16_bits(li.q), **kw)
+    d = O.decode(oc, W.bf16_bits(li.q), **kw)
+    if sel is not None:
+        bias = d.logg if (w.scorer == "gate" and w.gate_position != "off") else None
+        o, l = O.attend(oc, W.bf16_bits(li.q), sel[0], sel[1], w.scale, bias)
+        d = O.Decoded(d.score, np.asarray(sel[0]), np.asarray(sel[1]), d.logg, o, l)
+    return d
 
 
 def check_selection(ref: O.Decoded, sel_idx: np.ndarray, sel_cnt: np.ndarray, oc: O.Cache, w: W.Workload):

@@ -170,3 +170,45 @@ def test_rejects_bad_fold_gate_arguments_on_host():
               sba.sba_gate(0x100, 0x200, 257)):
         assert lib.sba_fold_gate(ctypes.byref(g), 0x1000, None) == E
     assert lib.sba_fold_gate(ctypes.byref(sba.sba_gate(0x100, 0x200, 128)), None, None) == E
+
+
+def test_rejects_bad_gate_variant_fields_on_host():
+    """log_gate and gate_act take their documented values, and are 0 for the Quest scorer."""
+    E = sba.SBA_ERR_INVALID_ARG
+    c = _cache(kg=0x9000)
+    assert _step(c, p=sba.select_params(16, 2, 0, 0, 0, 1, 3, 0), gate_A=0xa000) == E
+    assert _step(c, p=sba.select_params(16, 2, 0, 0, 0, 1, 1, 3), gate_A=0xa000) == E
+    assert _step(c, p=sba.select_params(16, 2, 0, 0, 0, 1, -1, 0), gate_A=0xa000) == E
+    assert _step(_cache(), p=sba.select_params(16, 2, 0, 0, 0, 0, 1, 0)) == E   # Quest has no log-gate
+    assert _step(_cache(), p=sba.select_params(16, 2, 0, 0, 0, 0, 0, 2)) == E
+
+
+def test_rejects_bad_multi_token_arguments_on_host():
+    lib = sba.load()
+    E = sba.SBA_ERR_INVALID_ARG
+    c = _cache()
+    p = sba.select_params(16, 2, 0, 0, 0, 0)
+    ssm = lib.sba_score_select_multi
+    ws = 0x100000
+    assert ssm(ctypes.byref(c), 0x5000, 0, ctypes.byref(p), 0x6000, 0x7000, 16, ws, 1 << 30, None) == E   # M = 0
+    assert ssm(ctypes.byref(c), 0x5000, 1025, ctypes.byref(p), 0x6000, 0x7000, 16, ws, 1 << 30, None) == E
+    assert ssm(ctypes.byref(c), 0x5008, 4, ctypes.byref(p), 0x6000, 0x7000, 16, ws, 1 << 30, None) == E
+    assert ssm(ctypes.byref(c), 0x5000, 4, ctypes.byref(p), 0x6000, 0x7000, 16, None, 0, None) == \
+        sba.SBA_ERR_WORKSPACE
+    gate = sba.select_params(16, 2, 0, 0, 0, 1, 1, 0)
+    assert ssm(ctypes.byref(_cache(kg=0x9000)), 0x5000, 4, ctypes.byref(gate), 0x6000, 0x7000, 16, ws, 1 << 30,
+               None) == sba.SBA_ERR_UNSUPPORTED                                    # Quest only
+    sdm = lib.sba_sparse_decode_multi
+    assert sdm(ctypes.byref(c), 0x5000, 0, 0x6000, 0x7000, 16, 0.088, 2, 0x8000, 0x9000, None) == E
+    assert sdm(ctypes.byref(c), 0x5000, 4, None, 0x7000, 16, 0.088, 2, 0x8000, 0x9000, None) == E
+    assert sdm(ctypes.byref(c), 0x5000, 4, 0x6000, 0x7000, 16, 0.0, 2, 0x8000, 0x9000, None) == E
+    assert sdm(ctypes.byref(c), 0x5000, 4, 0x6000, 0x7000, 16, 0.088, 0, 0x8000, 0x9000, None) == E
+    rect = lib.sba_rectify
+    assert rect(ctypes.byref(c), 0x5000, 0x1000, 0x2000, 0, 0.088, 2, 0x8000, 0x9000, None) == E
+    assert rect(ctypes.byref(c), 0x5000, 0x1000, 0x2000, 129, 0.088, 2, 0x8000, 0x9000, None) == \
+        sba.SBA_ERR_UNSUPPORTED                                                    # window beyond the ring
+    assert rect(ctypes.byref(c), 0x5000, None, 0x2000, 32, 0.088, 2, 0x8000, 0x9000, None) == E
+    assert rect(ctypes.byref(c), 0x5000, 0x1008, 0x2000, 32, 0.088, 2, 0x8000, 0x9000, None) == E
+    assert lib.sba_multi_row_groups(ctypes.byref(c), 32) == (32 * c.H_q // c.H_kv + 127) // 128
+    outer = lib.sba_sparse_decode_outer
+    assert outer(ctypes.byref(c), 0x5000, 0x6000, 0x7000, None, 16, 0.088, 2, 0x8000, 0x9000, None) == E  # needs g
