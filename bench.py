@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per context in SWEEP_CONTEXTS for each shape in SWEEP_SHAPES")
     ap.add_argument("--cpu-threads", type=int, default=0, help="threads of the all-cores oracle (0 = affinity)")
+    ap.add_argument("--prefetch", default="off", choices=["on", "off"],
+                    help="on: after each layer's step, an L2 prefetch of the next layer's descriptors")
     return ap.parse_args()
 
 
@@ -427,9 +429,13 @@ def native(args, rank, world, local, w=None, sweep=False):
                 "kernels": "mq_decode_kernel<dense> + combine_kernel per layer (one CUDA graph)"}
         del rgraph
 
+    prefetch = args.prefetch == "on"
+
     def step():
-        for L in layers:
+        for i, L in enumerate(layers):
             layer_step(w, L, p, pos, path=args.path)
+            if prefetch:  # the next layer's descriptors (the first layer's, for the next step)
+                sba.sba_prefetch_descriptors(layers[(i + 1) % n_layers]["c"])
 
     graph = capture(step)
     ms, clk = time_graph(graph, args.steps, args.warmup, flush_buf, world, local)
@@ -519,6 +525,8 @@ def native(args, rank, world, local, w=None, sweep=False):
                 else:
                     layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i], path=args.path)
                     od[i].copy_(L["bufs"].out)
+                if prefetch:
+                    sba.sba_prefetch_descriptors(layers[(i + 1) % n_layers]["c"])
             oh.copy_(od, non_blocking=True)
 
         for _ in range(2):
@@ -582,6 +590,8 @@ def native(args, rank, world, local, w=None, sweep=False):
                    f"{step_bytes / 1e6:.0f} MB" if flush else
                    f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step vs {l2 / 1e6:.0f} MB L2"),
             "graph": "one CUDA graph per step, programmatic dependent launch between kernels",
+            "prefetch": ("an L2 prefetch of the next layer's descriptors after each layer's step" if prefetch
+                         else "none"),
             "path": ("one fused sba_decode_step launch per layer (thread-block clusters)" if args.path == "fused"
                      else "five C-ABI calls per layer"),
             "parallelism": f"replicas x{world} (independent batches, no collective)",
@@ -589,7 +599,7 @@ def native(args, rank, world, local, w=None, sweep=False):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": KERNELS_PER_LAYER[args.path] * n_layers * args.steps,
+        "gpu_launches": (KERNELS_PER_LAYER[args.path] + (1 if prefetch else 0)) * n_layers * args.steps,
         "clocks": clk,
     }
     if rect is not None:

@@ -234,6 +234,16 @@ int sba_rectify(const sba_cache* c, const void* q, const void* k_new, const void
                                            num_splits, o_part, lse_part, static_cast<cudaStream_t>(stream)));
 }
 
+int sba_prefetch_descriptors(const sba_cache* c, void* stream) {
+    const int rc = check_cache(c);
+    if (rc != SBA_OK) return rc;
+    if (!c->desc && !c->kg) return SBA_ERR_INVALID_ARG;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SBA_ERR_CUDA;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return after_launch(launch_prefetch_descriptors(*c, sms, static_cast<cudaStream_t>(stream)));
+}
+
 int sba_combine(const float* o_part, const float* lse_part, int32_t B, int32_t H_q, int32_t num_splits, int32_t d,
                 void* out, int32_t out_dtype, float* lse_out, void* stream) {
     if (!o_part || !lse_part || !out || B < 1 || H_q < 1 || num_splits < 1) return SBA_ERR_INVALID_ARG;
