@@ -62,8 +62,8 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per context in SWEEP_CONTEXTS for each shape in SWEEP_SHAPES")
     ap.add_argument("--cpu-threads", type=int, default=0, help="threads of the all-cores oracle (0 = affinity)")
-    ap.add_argument("--prefetch", default="off", choices=["on", "off"],
-                    help="on: after each layer's step, an L2 prefetch of the next layer's descriptors")
+    ap.add_argument("--multi", type=int, default=0,
+                    help="M > 0: time M query tokens per sequence sharing one selection (Quest workloads)")
     return ap.parse_args()
 
 
@@ -429,13 +429,9 @@ def native(args, rank, world, local, w=None, sweep=False):
                 "kernels": "mq_decode_kernel<dense> + combine_kernel per layer (one CUDA graph)"}
         del rgraph
 
-    prefetch = args.prefetch == "on"
-
     def step():
-        for i, L in enumerate(layers):
+        for L in layers:
             layer_step(w, L, p, pos, path=args.path)
-            if prefetch:  # the next layer's descriptors (the first layer's, for the next step)
-                sba.sba_prefetch_descriptors(layers[(i + 1) % n_layers]["c"])
 
     graph = capture(step)
     ms, clk = time_graph(graph, args.steps, args.warmup, flush_buf, world, local)
@@ -525,8 +521,6 @@ def native(args, rank, world, local, w=None, sweep=False):
                 else:
                     layer_step(w, L, p, pos, q=qd[i], k_new=kd[i], v_new=vd[i], path=args.path)
                     od[i].copy_(L["bufs"].out)
-                if prefetch:
-                    sba.sba_prefetch_descriptors(layers[(i + 1) % n_layers]["c"])
             oh.copy_(od, non_blocking=True)
 
         for _ in range(2):
@@ -590,8 +584,6 @@ def native(args, rank, world, local, w=None, sweep=False):
                    f"{step_bytes / 1e6:.0f} MB" if flush else
                    f"inputs larger than L2: {step_bytes / 1e6:.0f} MB per step vs {l2 / 1e6:.0f} MB L2"),
             "graph": "one CUDA graph per step, programmatic dependent launch between kernels",
-            "prefetch": ("an L2 prefetch of the next layer's descriptors after each layer's step" if prefetch
-                         else "none"),
             "path": ("one fused sba_decode_step launch per layer (thread-block clusters)" if args.path == "fused"
                      else "five C-ABI calls per layer"),
             "parallelism": f"replicas x{world} (independent batches, no collective)",
@@ -599,7 +591,7 @@ def native(args, rank, world, local, w=None, sweep=False):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (KERNELS_PER_LAYER[args.path] + (1 if prefetch else 0)) * n_layers * args.steps,
+        "gpu_launches": KERNELS_PER_LAYER[args.path] * n_layers * args.steps,
         "clocks": clk,
     }
     if rect is not None:
@@ -611,6 +603,76 @@ def native(args, rank, world, local, w=None, sweep=False):
         out["rectify"] = rect
     del graph
     return out
+
+
+def native_multi(args, rank, world, local):
+    """M query tokens per sequence sharing one selection (sba_score_select_multi +
+    sba_sparse_decode_multi + sba_combine per layer, one CUDA graph per step); counted bytes
+    as the single-token step (one selection per group reads the same blocks)."""
+    import torch
+
+    from block_sparse_gqa_min_b200 import sba
+    from block_sparse_gqa_min_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sba.load()
+    w = workload_of(args)
+    if w.scorer != "quest":
+        raise SystemExit("--multi: Quest workloads only")
+    M = args.multi
+    n_layers = args.layers or w.layers
+    seed = rank_seed(args.seed, rank)
+    lay = W.make_layout(w, seed, device=dev)
+    layers, p, pos = build_layers(w, lay, seed, n_layers, dev)
+    c0 = layers[0]["c"]
+    n_max = layers[0]["bufs"].sel_idx.shape[-1]
+    rg = sba.sba_multi_row_groups(c0, M)
+    S = max(1, min(n_max, torch.cuda.get_device_properties(dev).multi_processor_count // (w.B * w.H_kv * rg)))
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed * 7 + M)
+    qs = [torch.randn((w.B, M, w.H_q, w.d), generator=g, device=dev).to(torch.bfloat16) for _ in range(n_layers)]
+    o_part = torch.empty((w.B, M, w.H_q, S, w.d), dtype=torch.float32, device=dev)
+    lse_part = torch.empty((w.B, M, w.H_q, S), dtype=torch.float32, device=dev)
+    out = torch.empty((w.B, M * w.H_q, w.d), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, M * w.H_q), dtype=torch.float32, device=dev)
+
+    def step():
+        for L, q in zip(layers, qs):
+            b = L["bufs"]
+            sba.sba_score_select_multi(L["c"], q, p, b.sel_idx, b.sel_cnt, b.ws)
+            sba.sba_sparse_decode_multi(L["c"], q, b.sel_idx, b.sel_cnt, w.scale, o_part, lse_part)
+            sba.sba_combine(o_part, lse_part, out, lse)
+
+    graph = capture(step)
+    lens = lay.seq_lens.cpu().tolist()
+    step_bytes = counted_bytes(w, lens, lambda N: sba.sba_num_selected(N, p)) * n_layers
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = (torch.empty((512 * 1024 * 1024 // 4,), dtype=torch.float32, device=dev)
+                 if step_bytes < 4 * l2 else None)
+    ms, clk = time_graph(graph, args.steps, args.warmup, flush_buf, world, local)
+    ms_max = max_over_ranks(ms, world, dev)
+    hbm, peak_kind = peaks()
+    gbs = job_gbs(step_bytes, world, ms_max)
+    status = [int(L["c"].status.item()) for L in layers]
+    if any(status):
+        raise RuntimeError(f"device status bits set: {status}")
+    del graph
+    return {
+        "metric": METRIC + f" ({M} query tokens per sequence sharing one selection)",
+        "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(ms_max, 4), "us_per_step": round(ms_max * 1e3, 1),
+        "us_per_layer": round(ms_max * 1e3 / n_layers, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "query_tokens": M, "batch": w.B, "layers": n_layers, "H_q": w.H_q,
+                   "H_kv": w.H_kv, "block": w.b, "context": [min(lens), max(lens)],
+                   "blocks_selected_per_group": n_max, "num_splits": S, "row_groups": rg,
+                   "counted_bytes_per_step": step_bytes,
+                   "graph": "score_select_multi + sparse_decode_multi + combine per layer, one CUDA graph"},
+        "roofline": {"bound": "hbm", "kernel": "step", "achieved": round(gbs / world, 1), "peak": hbm,
+                     "unit": "GB/s", "frac": round(gbs / world / hbm, 4), "peak_source": peak_kind},
+        "gpu_launches": 3 * n_layers * args.steps, "clocks": clk,
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -841,7 +903,11 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
-    if args.sweep:
+    if args.multi:
+        out = native_multi(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    elif args.sweep:
         # the "vs context" curve: every context at the R1-7B and Qwen3-14B shapes, one line each
         from block_sparse_gqa_min_b200 import workloads as W
 

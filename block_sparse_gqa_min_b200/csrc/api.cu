@@ -230,18 +230,8 @@ int sba_rectify(const sba_cache* c, const void* q, const void* k_new, const void
     if (rc != SBA_OK) return rc;
     if (f > kMaxRectifyTokens) return SBA_ERR_UNSUPPORTED;
     if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SBA_ERR_INVALID_ARG;
-    return after_launch(launch_multi_query(*c, q, f, nullptr, nullptr, 0, k_new, v_new, true, softmax_scale,
-                                           num_splits, o_part, lse_part, static_cast<cudaStream_t>(stream)));
-}
-
-int sba_prefetch_descriptors(const sba_cache* c, void* stream) {
-    const int rc = check_cache(c);
-    if (rc != SBA_OK) return rc;
-    if (!c->desc && !c->kg) return SBA_ERR_INVALID_ARG;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SBA_ERR_CUDA;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return after_launch(launch_prefetch_descriptors(*c, sms, static_cast<cudaStream_t>(stream)));
+    return after_launch(launch_rectify_tc(*c, q, f, k_new, v_new, softmax_scale, num_splits, o_part, lse_part,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 int sba_combine(const float* o_part, const float* lse_part, int32_t B, int32_t H_q, int32_t num_splits, int32_t d,

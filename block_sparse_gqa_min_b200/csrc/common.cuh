@@ -308,13 +308,6 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// fp32 -> tf32 (round to nearest, ties away from zero); the low 13 bits are zero.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
 // D += A B on tensor cores, tf32 inputs, fp32 accumulate (m16n8k8).
 __device__ __forceinline__ void mma_tf32_1688(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
     asm volatile(

@@ -677,8 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 } else {
                     // u = q . kg on tensor cores: tiles of 16 blocks (rows) x 8 heads (columns);
-                    // kg = hi + lo (hi = kg rounded to tf32, lo = the exact remainder, read by the MMA
-                    // truncated to tf32: about 21 bits of kg in all); four
+                    // kg = hi + lo (hi = kg truncated to tf32 by a bit mask -- a full-rate logic op,
+                    // where a rounding conversion runs at a fraction of the issue rate -- and lo = the
+                    // exact remainder, read by the MMA truncated to tf32: about 21 bits of kg); four
                     // accumulators per tile (channel half x hi/lo) keep the MMA chains short, and
                     // a warp's tiles of the stage run interleaved when registers allow
                     constexpr int kTl = (kIt == 2 && NTq == 1) ? 2 : 1;
@@ -709,8 +710,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                         e ? x1.w : x1.y};
                                     uint32_t hi[4], lo[4];
 #pragma unroll
-                                    for (int u = 0; u < 4; ++u) {  // (the MMA reads lo's top 19 bits)
-                                        hi[u] = to_tf32(v[u]);
+                                    for (int u = 0; u < 4; ++u) {  // (the MMA reads the top 19 bits of each)
+                                        hi[u] = __float_as_uint(v[u]) & 0xffffe000u;  // v truncated to tf32
                                         lo[u] = __float_as_uint(v[u] - __uint_as_float(hi[u]));
                                     }
                                     const int ah = (p >> 2) * 2;  // accumulator pair of this channel half
@@ -758,39 +759,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------- phase 2: distributed selection ----------------
     if (kScorer == SBA_SCORER_GATE) {
-        // softmax gates: per-head (max, sum exp(u - max)) over this CTA's scored blocks, pushed to
-        // every CTA; sigmoid and unnormalised gates need no normaliser (lse = 0 below)
+        // softmax gates: per-head (max, sum exp(u - max)) over this CTA's scored blocks, one warp
+        // per head, pushed to every CTA; sigmoid and unnormalised gates need no normaliser (lse = 0
+        // below).  Exponentials are exp2 of log2(e)-scaled arguments (one special-function op each).
         const bool softmax_gate = a.p.gate_act == SBA_GATE_SOFTMAX;
-        for (int g = warp; softmax_gate && g < G; g += kThreads / 32) {
-            float m = -INFINITY;
-            for (int i = lane; i < js1 - j0; i += 32) m = fmaxf(m, u_s[g * ustride + i]);
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            float z = 0.f;
-            if (m > -INFINITY)
-                for (int i = lane; i < js1 - j0; i += 32) z += expf(u_s[g * ustride + i] - m);
+        if (softmax_gate) {
+            for (int g = warp; g < G; g += kThreads / 32) {
+                float m = -INFINITY;
+                for (int i = lane; i < js1 - j0; i += 32) m = fmaxf(m, u_s[g * ustride + i]);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-            for (int p = lane; p < C; p += 32) {
-                st_peer_f32(peer_addr(&mz_all[r * G + g][0], p), m);
-                st_peer_f32(peer_addr(&mz_all[r * G + g][1], p), z);
-            }
-        }
-        if (softmax_gate) cluster_sync();  // gate round: every CTA's softmax partials pushed
-        if (tid < G && !softmax_gate) lse_s[tid] = 0.f;
-        if (tid < G && softmax_gate) {
-            float M = -INFINITY;
-            for (int p = 0; p < C; ++p) M = fmaxf(M, mz_all[p * G + tid][0]);
-            float Z = 0.f;
-            if (M > -INFINITY)
-                for (int p = 0; p < C; ++p) {
-                    const float m = mz_all[p * G + tid][0];
-                    if (m > -INFINITY) Z += mz_all[p * G + tid][1] * expf(m - M);
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                float z = 0.f;
+                if (m > -INFINITY)
+                    for (int i = lane; i < js1 - j0; i += 32) z += exp2f((u_s[g * ustride + i] - m) * kLog2e);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                for (int p = lane; p < C; p += 32) {
+                    st_peer_f32(peer_addr(&mz_all[r * G + g][0], p), m);
+                    st_peer_f32(peer_addr(&mz_all[r * G + g][1], p), z);
                 }
-            lse_s[tid] = M > -INFINITY ? M + logf(Z) : -INFINITY;
+            }
+            cluster_sync();  // gate round: every CTA's softmax partials pushed
+            // LSE of head g by warp g: lane p reads CTA p's pair (C <= 16 lanes)
+            for (int g = warp; g < G; g += kThreads / 32) {
+                const float m = lane < C ? mz_all[lane * G + g][0] : -INFINITY;
+                const float z = lane < C ? mz_all[lane * G + g][1] : 0.f;
+                float M = m;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+                float Z = (M > -INFINITY && m > -INFINITY) ? z * exp2f((m - M) * kLog2e) : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+                if (lane == 0) lse_s[g] = M > -INFINITY ? M + logf(Z) : -INFINITY;
+            }
+        } else if (tid < G) {
+            lse_s[tid] = 0.f;
         }
         __syncthreads();
         // group score of my ranked blocks: sum over the group of g (softmax: exp(u - LSE); raw:
@@ -807,10 +810,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sc[2] += gate_of(u4.z, 0.f, SBA_GATE_SIGMOID);
                     sc[3] += gate_of(u4.w, 0.f, SBA_GATE_SIGMOID);
                 } else {
-                    sc[0] += expf(u4.x - lse_s[g]);
-                    sc[1] += expf(u4.y - lse_s[g]);
-                    sc[2] += expf(u4.z - lse_s[g]);
-                    sc[3] += expf(u4.w - lse_s[g]);
+                    sc[0] += exp2f((u4.x - lse_s[g]) * kLog2e);
+                    sc[1] += exp2f((u4.y - lse_s[g]) * kLog2e);
+                    sc[2] += exp2f((u4.z - lse_s[g]) * kLog2e);
+                    sc[3] += exp2f((u4.w - lse_s[g]) * kLog2e);
                 }
             }
             uint32_t kk[4];

@@ -109,7 +109,6 @@ _SIGS = {
                                 ctypes.c_int),
     "sba_multi_row_groups": ([ctypes.POINTER(sba_cache), _I], _I),
     "sba_rectify": ([ctypes.POINTER(sba_cache), _P, _P, _P, _I, ctypes.c_float, _I, _P, _P, _P], ctypes.c_int),
-    "sba_prefetch_descriptors": ([ctypes.POINTER(sba_cache), _P], ctypes.c_int),
     "sba_combine": ([_P, _P, _I, _I, _I, _I, _P, _I, _P, _P], ctypes.c_int),
     "sba_fold_gate": ([ctypes.POINTER(sba_gate), _P, _P], ctypes.c_int),
     "sba_static_scratch_bytes": ([], ctypes.c_size_t),
@@ -327,11 +326,6 @@ def sba_rectify(c: Cache, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Ten
     num_splits = int(lse_part.shape[-1])
     _check(load().sba_rectify(ctypes.byref(c.struct()), _ptr(q), _ptr(k_new), _ptr(v_new), f, float(softmax_scale),
                               num_splits, _ptr(o_part), _ptr(lse_part), _stream(stream)), "sba_rectify")
-
-
-def sba_prefetch_descriptors(c: Cache, stream=None):
-    """An L2 prefetch hint for the layer's descriptors (writes nothing)."""
-    _check(load().sba_prefetch_descriptors(ctypes.byref(c.struct()), _stream(stream)), "sba_prefetch_descriptors")
 
 
 def sba_combine(o_part: torch.Tensor, lse_part: torch.Tensor, out: torch.Tensor,

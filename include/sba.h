@@ -318,20 +318,6 @@ int32_t sba_multi_row_groups(const sba_cache *c, int32_t M);
 int sba_rectify(const sba_cache *c, const void *q, const void *k_new, const void *v_new, int32_t f,
                 float softmax_scale, int32_t num_splits, float *o_part, float *lse_part, void *stream);
 
-/* Ask the L2 cache to fetch the block descriptors of a layer (c->desc, or
- * c->kg when desc is NULL: every valid block of every sequence) ahead of its
- * decode step.  The scan of every descriptor is the part of a step that
- * depends on the cache alone, not on the query ("Rectified Sparse Attention
- * ...", Key points: the 1/b term of the per-step memory); enqueued between
- * the steps of two layers, the fetch of the second layer's descriptors
- * overlaps the first layer's selection, attention and merge.
- * A hint: it writes nothing and changes no result.  The kernel starts while
- * the kernel before it in the stream is still running (programmatic
- * dependent launch) and completes only after that kernel has completed, so
- * the order the stream gives every later kernel is unchanged.  It reads
- * seq_lens and the block table before that point, to size the fetch only. */
-int sba_prefetch_descriptors(const sba_cache *c, void *stream);
-
 /* Size in bytes of the static scratch behind sba_score_select_static (8 MiB). */
 size_t sba_static_scratch_bytes(void);
 
