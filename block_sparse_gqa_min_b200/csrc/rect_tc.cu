@@ -8,30 +8,34 @@
 // key and value tile, this is a dense contraction: 128 query rows against each
 // 64-token tile, the shape the tensor cores take whole.
 //
-// One CTA per (split, KV head x row group of 128 query rows, sequence); 192
+// One CTA per (split, KV head x row group of 128 query rows, sequence); 320
 // threads:
-//  - warp 4 (producer) streams each block in 64-token stages (K0 K1 V0 V1: four
+//  - warp 8 (producer) streams each block in 64-token stages (K0 K1 V0 V1: four
 //    2-D TMA loads of 64 rows x 128 B, 128-byte swizzle, no multicast) into a
 //    ring of 32 KB stages.  Before a block the window touches is loaded, it
 //    writes the window's K/V rows of that block into the cache (a proxy fence
 //    orders them ahead of the tile load); after its last fill it recomputes the
-//    Quest min/max of those blocks from the staged K rows.  Rows past len are
-//    zeroed in the stage before anyone reads it.
-//  - warp 5 (MMA) allocates 256 TMEM columns and, one thread issuing, runs per
-//    stage S = Q K^T (M 128 rows, N 64 tokens, K 128 channels: eight
-//    tcgen05.mma kind::f16, bf16 in, fp32 accumulate into TMEM columns 0-63),
-//    then, once the softmax warps have written P, O += P_hi V + P_lo V (M 128,
-//    N 128 channels, K 64 tokens; V read MN-major straight from the TMA tile)
-//    into TMEM columns 128-255.  tcgen05.commit signals S, O and the stage's
-//    release on mbarriers.
-//  - warps 0-3 (softmax): thread r owns query row r = TMEM lane r.  It reads its
-//    row of S (tcgen05.ld 32x32b.x64), applies the causal limit (t <= len - f + i
-//    for token i) and the scale, keeps an online softmax whose exponent offset
-//    moves only when the row maximum grows by more than 2^8 (then O's row is
-//    rescaled in TMEM; otherwise exponentials stay below 2^8), and writes P as
-//    bf16 hi + lo parts (about 16 mantissa bits) into the 128-byte-swizzled A
-//    tile of the next MMA.  At the end it reads its O row, normalises it and
-//    writes the split's O and LSE ([B][f][H_q][S][d], [B][f][H_q][S]).
+//    Quest min/max of those blocks from their keys.  Rows past len are zeroed in
+//    the stage before anyone reads it.
+//  - warp 9 (MMA) allocates 256 TMEM columns and, one thread issuing, runs
+//    S = Q K^T for each stage (M 128 rows, N 64 tokens, K 128 channels: eight
+//    tcgen05.mma kind::f16, bf16 in, fp32 accumulate) into one of two TMEM S
+//    buffers (columns 0-63, 64-127), so the next stage's S is computed while
+//    the softmax works on this one; then, once P is written,
+//    O += P_hi V + P_lo V (M 128, N 128 channels, K 64 tokens; V read MN-major
+//    straight from the TMA tile) into TMEM columns 128-255.  tcgen05.commit
+//    signals S, O and the stage's release on mbarriers.
+//  - warps 0-7 (softmax): query row r = TMEM lane r is shared by warps r/32
+//    and r/32 + 4, each owning 32 of the stage's 64 columns.  A thread reads
+//    its half row of S (tcgen05.ld 32x32b.x32), applies the causal limit
+//    (t <= len - f + i for token i) and the scale, agrees on the row maximum
+//    with its partner through shared memory, keeps an online softmax whose
+//    exponent offset moves only when the row maximum grows by more than 2^8
+//    (then O's row is rescaled in TMEM; otherwise exponentials stay below
+//    2^8), and writes its half of P as bf16 hi + lo parts (about 16 mantissa
+//    bits) into one of two 128-byte-swizzled A tiles.  At the end it reads its
+//    64 columns of O, normalises them and writes the split's O and LSE
+//    ([B][f][H_q][S][d], [B][f][H_q][S]).
 // Every wait is bounded: a wait that runs out reports SBA_DEV_TIMEOUT and the
 // roles stop, and TMEM is released on every path.
 #include <cuda.h>
@@ -49,16 +53,16 @@ bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);  // decod
 namespace {
 
 constexpr int kRtRows = 128;               // query rows per CTA: the MMA's M
-constexpr int kRtStages = 4;               // 64-token K/V stages
+constexpr int kRtStages = 3;               // 64-token K/V stages (with the two P buffers, all that fits)
 constexpr int kRtStage = 32768;
 constexpr int kRtHalf = 8192;              // 64 rows x 128 B
-constexpr int kRtThreads = 192;            // warps 0-3 softmax, 4 producer, 5 MMA
-constexpr int kProdWarp = 4, kMmaWarp = 5;
+constexpr int kRtThreads = 320;            // warps 0-7 softmax, 8 producer, 9 MMA
+constexpr int kProdWarp = 8, kMmaWarp = 9;
 constexpr int kOffQ = 0;                   // 2 x 16 KB: 128 rows x 64 channels, K-major, 128-B swizzle
-constexpr int kOffP = 32768;               // P hi (16 KB) then P lo (16 KB): 128 rows x 64 tokens
-constexpr int kOffRing = 65536;
+constexpr int kOffP = 32768;               // two P buffers of 32 KB: hi (16 KB) then lo, 128 rows x 64 tokens
+constexpr int kOffRing = 98304;
 constexpr int kRtSmem = kOffRing + kRtStages * kRtStage + 1024;
-constexpr uint32_t kTmemCols = 256;        // S: columns 0-63; O: 128-255
+constexpr uint32_t kTmemCols = 256;        // S buffers: columns 0-63 and 64-127; O: 128-255
 constexpr uint32_t kColS = 0, kColO = 128;
 
 struct RtArgs {
@@ -118,6 +122,29 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
 #pragma unroll
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 2^x by the special-function unit (flushes results below 2^-126 to zero, which no softmax
+// weight here can reach with any effect)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
 __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -167,8 +194,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     constexpr int kSub = kBlk / 64;
     extern __shared__ uint8_t dyn_raw[];
     uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t kv_full[kRtStages], kv_empty[kRtStages], zbar, s_full, p_full, pv_done, fin;
+    __shared__ uint64_t kv_full[kRtStages], kv_empty[kRtStages], zbar, s_full[2], p_full[2], pv_done[2], fin;
     __shared__ uint32_t tmem_base;
+    __shared__ float xmax[2][2][kRtRows];  // [stage parity][column half][row]: partial row maxima
+    __shared__ float xl[2][kRtRows];       // [column half][row]: partial row sums at the end
 
     const sba_cache& c = a.c;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,9 +212,11 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             mbar_init(&kv_empty[i], 1);
         }
         mbar_init(&zbar, 1);
-        mbar_init(&s_full, 1);
-        mbar_init(&p_full, 4);
-        mbar_init(&pv_done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[b], 8);  // one arrival per softmax warp
+            mbar_init(&pv_done[b], 1);
+        }
         mbar_init(&fin, 1);
         fence_mbar_init();
     }
@@ -214,20 +245,23 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     const int tb0 = appends ? pos0 / kBlk : N;
     const int i0 = (int)((int64_t)N * sp / a.num_splits), i1 = (int)((int64_t)N * (sp + 1) / a.num_splits);
     const int nfill = (i1 - i0) * kSub;
-    auto fill_valid = [&](int f) {  // tokens of fill f below len (0: the fill is skipped by every role)
+    auto fill_valid = [&](int f) {  // tokens of fill f below len
         const int j = i0 + f / kSub, sb = f % kSub;
         return min(64, max(0, len - j * kBlk - 64 * sb));
     };
+    // only the last block's second half can be empty, and it is the last fill of its share: the
+    // processed fills are fills 0 .. nproc-1 for every role
+    const int nproc = (nfill > 0 && fill_valid(nfill - 1) == 0) ? nfill - 1 : nfill;
 
     // the query rows of this CTA into the K-major, 128-byte-swizzled A tile (zero past the group's rows)
-    if (warp < 4) {
-        const int r = tid, gr = row0 + r;
+    if (warp < 8) {
+        const int r = tid & 127, half = tid >> 7, gr = row0 + r;
         const __nv_bfloat16* qrow =
             gr < R ? a.q + (((int64_t)s * a.M + gr / G) * c.H_q + h * G + gr % G) * kHeadDim : nullptr;
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-            const uint4 v = qrow ? __ldg(reinterpret_cast<const uint4*>(qrow) + ch) : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(dyn + kOffQ + (ch >> 3) * 16384 + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = v;
+        for (int cc = 0; cc < 8; ++cc) {
+            const uint4 v = qrow ? __ldg(reinterpret_cast<const uint4*>(qrow) + 8 * half + cc) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(dyn + kOffQ + half * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();
     }
@@ -240,11 +274,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     if (warp == kProdWarp) {
         // ------------------------------ producer ------------------------------
         uint32_t zpar = 0;
-        int q = 0;  // processed fills (ring slots)
-        for (int f = 0; f < nfill && alive; ++f) {
-            const int vf = fill_valid(f);
-            if (vf == 0) continue;
-            const int i = i0 + f / kSub, sb = f % kSub, j = i;
+        for (int q = 0; q < nproc && alive; ++q) {
+            const int vf = fill_valid(q);
+            const int i = i0 + q / kSub, sb = q % kSub, j = i;
             const int st = q % kRtStages;
             if (q >= kRtStages) {
                 if (lane == 0) alive = mbar_wait(&kv_empty[st], ((q / kRtStages) - 1) & 1, c.status);
@@ -259,7 +291,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&kv_full[st]);
-                ++q;
                 continue;
             }
             if (appends && sb == 0 && j >= tb0) {
@@ -299,47 +330,36 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 if (lane == 0) mbar_arrive(&kv_full[st]);
                 if (!ok) alive = false;
             }
-            ++q;
         }
-        // the Quest descriptors of the blocks the window touched, from their staged K rows (the
-        // last fills of this share, still in the ring: nothing is loaded after them)
-        const int nproc = q;
+        // the Quest descriptors of the blocks the window touched that lie in this share, recomputed
+        // from all of each block's valid keys in global memory (the window's rows were written above
+        // by this warp; at most three blocks per head)
         if (appends && c.desc && rg == 0 && alive) {
-            for (int pq = max(0, nproc - kRtStages); pq < nproc; ++pq) {
-                // processed fill pq is fill pq (only the very last fill of a share can be skipped)
-                const int i = i0 + pq / kSub, sb = pq % kSub, j = i;
-                if (sb != 0 || j < tb0) continue;
+            __syncwarp();
+            for (int j = max(tb0, i0); j < min(N, i1); ++j) {
+                const int pg = (int)page_of(c, s, j, nullptr);
+                if (pg < 0) continue;
                 const int vb = min(kBlk, len - j * kBlk);
+                const uint4* krows = reinterpret_cast<const uint4*>(c.k) + ((int64_t)pg * c.H_kv + h) * kBlk * 16;
                 uint32_t mn[4], mx[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) mn[e] = 0x7f807f80u, mx[e] = 0xff80ff80u;
-                bool ok = true;
-                for (int sub = 0; sub < kSub && ok; ++sub) {
-                    const int ff = pq + sub, vs = min(64, vb - 64 * sub);
-                    if (vs <= 0 || ff >= nproc) break;
-                    if (lane == 0) ok = mbar_wait(&kv_full[ff % kRtStages], (ff / kRtStages) & 1, c.status);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    const uint8_t* kt = dyn + kOffRing + (size_t)(ff % kRtStages) * kRtStage;
-                    const int ck = lane & 15, cc = ck & 7;
-                    for (int t = lane >> 4; t < vs; t += 2) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(kt + (ck >> 3) * kRtHalf + t * 128 + ((cc ^ (t & 7)) << 4));
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                const int ck = lane & 15;  // 16-byte chunk (8 channels) of a row; lanes 16-31 take odd rows
+                for (int t = lane >> 4; t < vb; t += 2) {
+                    const uint4 w = krows[t * 16 + ck];
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            mn[e] = bmin2(mn[e], ws[e]);
-                            mx[e] = bmax2(mx[e], ws[e]);
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        mn[e] = bmin2(mn[e], ws[e]);
+                        mx[e] = bmax2(mx[e], ws[e]);
                     }
                 }
-                if (!ok) break;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     mn[e] = bmin2(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], 16));
                     mx[e] = bmax2(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
                 }
-                const int pg = (int)page_of(c, s, j, nullptr);
-                if (lane < 16 && pg >= 0) {
+                if (lane < 16) {
                     uint8_t* d = reinterpret_cast<uint8_t*>(c.desc) + ((int64_t)pg * c.H_kv + h) * 2 * kHeadDim * 2;
                     *reinterpret_cast<uint4*>(d + lane * 16) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
                     *reinterpret_cast<uint4*>(d + 2 * kHeadDim + lane * 16) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
@@ -350,46 +370,55 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // ------------------------------ MMA issue ------------------------------
         constexpr uint32_t kIdQK = umma_idesc(128, 64, false);
         constexpr uint32_t kIdPV = umma_idesc(128, 128, true);
-        const uint32_t sQ = smem_u32(dyn + kOffQ), sP = smem_u32(dyn + kOffP);
-        int q = 0;
+        const uint32_t sQ = smem_u32(dyn + kOffQ), sP0 = smem_u32(dyn + kOffP);
         bool issued = false;  // any MMA issued by this warp
-        for (int f = 0; f < nfill && alive; ++f) {
-            if (fill_valid(f) == 0) continue;
+        // S(q) = Q K(q)^T into S buffer q % 2; K = 128 channels in eight steps of 16 (32 bytes
+        // along the swizzled rows)
+        auto issue_qk = [&](int q) {
             const int st = q % kRtStages;
             if (lane == 0) alive = mbar_wait(&kv_full[st], (q / kRtStages) & 1, c.status);
             alive = __shfl_sync(0xffffffffu, alive, 0);
-            if (!alive) break;
+            if (!alive) return;
             tc_fence_after();
             const uint32_t sK = smem_u32(dyn + kOffRing + (size_t)st * kRtStage);
-            const uint32_t sV = sK + 2 * kRtHalf;
             if (lane == 0) {
-                // S = Q K^T: K = 128 channels in eight steps of 16 (32 bytes along the swizzled rows)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tm + kColS, umma_desc(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    umma_f16(tm + kColS + 64 * (q & 1), umma_desc(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                              umma_desc(sK + (kk >> 2) * kRtHalf + (kk & 3) * 32, 16, 1024), kIdQK, kk > 0);
-                umma_commit(&s_full);
+                umma_commit(&s_full[q & 1]);
             }
             issued = true;
             __syncwarp();
-            if (lane == 0) alive = mbar_wait(&p_full, q & 1, c.status);
+        };
+        if (nproc > 0) issue_qk(0);
+        for (int q = 0; q < nproc && alive; ++q) {
+            // the next stage's S overlaps this stage's softmax (its S buffer was read by the softmax of
+            // stage q - 1, whose P has been waited for)
+            if (q + 1 < nproc) {
+                issue_qk(q + 1);
+                if (!alive) break;
+            }
+            if (lane == 0) alive = mbar_wait(&p_full[q & 1], (q >> 1) & 1, c.status);
             alive = __shfl_sync(0xffffffffu, alive, 0);
             if (!alive) break;
             tc_fence_after();
+            const int st = q % kRtStages;
+            const uint32_t sV = smem_u32(dyn + kOffRing + (size_t)st * kRtStage) + 2 * kRtHalf;
+            const uint32_t sP = sP0 + (q & 1) * 32768;
             if (lane == 0) {
-                // O += P V: K = 64 tokens in four steps of 16 (two 8-row groups of the V tile each);
-                // V is MN-major: its two 64-channel halves are 8 KB apart
+                // O += P V: K = 64 tokens in four steps of 16 (two 8-row groups of the V tile each); V is
+                // MN-major, its two 64-channel halves 8 KB apart
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tm + kColO, umma_desc(sP + part * 16384 + kk * 32, 16, 1024),
                                  umma_desc(sV + kk * 2048, kRtHalf, 1024), kIdPV, (q > 0 || part > 0 || kk > 0));
-                umma_commit(&pv_done);
+                umma_commit(&pv_done[q & 1]);
                 umma_commit(&kv_empty[st]);
             }
             __syncwarp();
-            ++q;
         }
         // every MMA this warp issued has completed before TMEM can be released (also after a
         // wait that ran out)
@@ -400,73 +429,102 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------ softmax ------------------------------
-        const int r = tid;  // query row = TMEM lane
+        const int qd = warp & 3, hf = warp >> 2;  // lane quarter, column half
+        const int r = 32 * qd + lane;              // query row = TMEM lane
         const int gr = row0 + r;
         const int lim = gr < R ? pos0 + gr / G + 1 : 0;  // causal limit (exclusive)
-        const uint32_t lane_base = tm + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tm + ((uint32_t)(qd * 32) << 16);
         float m_used = -INFINITY, l = 0.f;
-        int q = 0;
-        for (int f = 0; f < nfill && alive; ++f) {
-            const int vf = fill_valid(f);
-            if (vf == 0) continue;
-            const int j = i0 + f / kSub, sb = f % kSub;
-            const int base = j * kBlk + 64 * sb;
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(&s_full, q & 1, c.status);
-            alive = __shfl_sync(0xffffffffu, ok, 0);
-            if (!alive) break;
-            tc_fence_after();
-            float sv[64];
-            tmem_ld64(lane_base + kColS, sv);
+        // (a wait that runs out turns this warp dead; a dead warp still takes every named barrier of the
+        // loop, so its partner never waits on it forever, and arrives on nothing)
+        for (int q = 0; q < nproc; ++q) {
+            const int vf = fill_valid(q);
+            const int j = i0 + q / kSub, sb = q % kSub;
+            const int base = j * kBlk + 64 * sb + 32 * hf;  // position of this half's first token
+            bool ok = alive;
+            if (ok) {
+                if (lane == 0) ok = mbar_wait(&s_full[q & 1], (q >> 1) & 1, c.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+            }
+            float sv[32];
             float mx = -INFINITY;
+            if (ok) {
+                tc_fence_after();
+                tmem_ld32(lane_base + kColS + 64 * (q & 1) + 32 * hf, sv);
+                const int nval = min(32, min(vf - 32 * hf, lim - base));  // valid columns of this half row
+                if (nval >= 32) {
 #pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                sv[t] = (t < vf && base + t < lim) ? sv[t] * a.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sv[t]);
+                    for (int t = 0; t < 32; ++t) sv[t] *= a.scale_log2;
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) sv[t] = t < nval ? sv[t] * a.scale_log2 : -INFINITY;
+                }
+                float m8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) m8[u] = fmaxf(fmaxf(sv[u], sv[u + 8]), fmaxf(sv[u + 16], sv[u + 24]));
+#pragma unroll
+                for (int u = 0; u < 4; ++u) m8[u] = fmaxf(m8[u], m8[u + 4]);
+                mx = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+            }
+            // the row maximum agreed with the partner warp (the other half of the row's columns)
+            xmax[q & 1][hf][r] = mx;
+            named_bar(1 + qd, 64);
+            mx = fmaxf(mx, xmax[q & 1][hf ^ 1][r]);
+            if (!ok) {
+                alive = false;
+                continue;
             }
             // the exponent offset moves only when the maximum grows by more than 2^8
             float alpha = 1.f;
             if (mx > -INFINITY && (m_used == -INFINITY || mx > m_used + 8.f)) {
-                alpha = m_used == -INFINITY ? 0.f : exp2f(m_used - mx);
+                alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mx);
                 m_used = mx;
                 l *= alpha;
             }
             const bool rescale = q > 0 && alpha != 1.f;
-            float lsum = 0.f;
-            uint32_t ph[32], pl[32];
+            uint32_t ph[16], pl[16];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int t = 0; t < 64; t += 2) {
-                const float p0 = m_used == -INFINITY ? 0.f : exp2f(sv[t] - m_used);
-                const float p1 = m_used == -INFINITY ? 0.f : exp2f(sv[t + 1] - m_used);
-                lsum += p0 + p1;
+            for (int t = 0; t < 32; t += 2) {
+                const float p0 = m_used == -INFINITY ? 0.f : ex2(sv[t] - m_used);
+                const float p1 = m_used == -INFINITY ? 0.f : ex2(sv[t + 1] - m_used);
+                ls[(t >> 1) & 3] += p0 + p1;
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-                const float2 hf = __bfloat1622float2(hi);
-                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                const float2 hfv = __bfloat1622float2(hi);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hfv.x, p1 - hfv.y);
                 ph[t / 2] = *reinterpret_cast<const uint32_t*>(&hi);
                 pl[t / 2] = *reinterpret_cast<const uint32_t*>(&lo);
             }
-            l += lsum;
-            // P and O are free once the previous O += P V has completed
-            if (q > 0) {
-                if (lane == 0) ok = mbar_wait(&pv_done, (q - 1) & 1, c.status);
-                alive = __shfl_sync(0xffffffffu, ok, 0);
-                if (!alive) break;
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            // this P buffer is free once O += P V of stage q - 2 has completed; O itself (to rescale)
+            // once that of stage q - 1 has
+            if (q >= 2) {
+                if (lane == 0) ok = mbar_wait(&pv_done[q & 1], ((q - 2) >> 1) & 1, c.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    alive = false;
+                    continue;
+                }
                 tc_fence_after();
             }
             if (__any_sync(0xffffffffu, rescale)) {
-                float ov[64];
-#pragma unroll
-                for (int hlf = 0; hlf < 2; ++hlf) {
-                    tmem_ld64(lane_base + kColO + 64 * hlf, ov);
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) ov[e] *= rescale ? alpha : 1.f;
-                    tmem_st64(lane_base + kColO + 64 * hlf, ov);
+                if (lane == 0) ok = mbar_wait(&pv_done[(q - 1) & 1], ((q - 1) >> 1) & 1, c.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    alive = false;
+                    continue;
                 }
-            }
-            uint8_t* prow = dyn + kOffP + r * 128;
+                tc_fence_after();
+                float ov[64];
+                tmem_ld64(lane_base + kColO + 64 * hf, ov);
 #pragma unroll
-            for (int cch = 0; cch < 8; ++cch) {
-                const int off = ((cch ^ (r & 7)) << 4);
+                for (int e = 0; e < 64; ++e) ov[e] *= rescale ? alpha : 1.f;
+                tmem_st64(lane_base + kColO + 64 * hf, ov);
+            }
+            uint8_t* prow = dyn + kOffP + (q & 1) * 32768 + r * 128;
+#pragma unroll
+            for (int cch = 0; cch < 4; ++cch) {
+                const int off = (((4 * hf + cch) ^ (r & 7)) << 4);
                 *reinterpret_cast<uint4*>(prow + off) = make_uint4(ph[4 * cch], ph[4 * cch + 1], ph[4 * cch + 2], ph[4 * cch + 3]);
                 *reinterpret_cast<uint4*>(prow + 16384 + off) =
                     make_uint4(pl[4 * cch], pl[4 * cch + 1], pl[4 * cch + 2], pl[4 * cch + 3]);
@@ -474,35 +532,35 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full);
-            ++q;
+            if (lane == 0) mbar_arrive(&p_full[q & 1]);
         }
-        // the split's normalised output of this row
-        float ov[2][64];
+        // the split's normalised output of this row: this warp's 64 channels
+        xl[hf][r] = l;
+        named_bar(1 + qd, 64);
+        const float lt = xl[0][r] + xl[1][r];
+        float ov[64];
         bool have = false;
-        if (alive && q > 0) {
+        if (alive && nproc > 0) {
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(&pv_done, (q - 1) & 1, c.status);
+            if (lane == 0) ok = mbar_wait(&pv_done[(nproc - 1) & 1], ((nproc - 1) >> 1) & 1, c.status);
             have = __shfl_sync(0xffffffffu, ok, 0);
             if (have) {
                 tc_fence_after();
-                tmem_ld64(lane_base + kColO, ov[0]);
-                tmem_ld64(lane_base + kColO + 64, ov[1]);
+                tmem_ld64(lane_base + kColO + 64 * hf, ov);
             }
         }
         if (gr < R) {
             const int ti = gr / G, g = gr % G;
             const int64_t orow = (((int64_t)s * a.M + ti) * c.H_q + h * G + g) * a.num_splits + sp;
-            float* dst = a.o_part + orow * kHeadDim;
-            const bool any = have && l > 0.f;
-            const float inv = any ? 1.f / l : 0.f;
+            float* dst = a.o_part + orow * kHeadDim + 64 * hf;
+            const bool any = have && lt > 0.f;
+            const float inv = any ? 1.f / lt : 0.f;
 #pragma unroll
-            for (int e = 0; e < 128; e += 4)
+            for (int e = 0; e < 64; e += 4)
                 *reinterpret_cast<float4*>(dst + e) =
-                    any ? make_float4(ov[e >> 6][e & 63] * inv, ov[e >> 6][(e & 63) + 1] * inv,
-                                      ov[e >> 6][(e & 63) + 2] * inv, ov[e >> 6][(e & 63) + 3] * inv)
+                    any ? make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
-            a.lse_part[orow] = any ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+            if (hf == 0) a.lse_part[orow] = any ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
         }
     }
     // every role is done with TMEM: the allocating warp releases it

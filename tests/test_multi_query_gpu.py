@@ -164,6 +164,8 @@ RECT_CASES = [
     (dict(H_q=8, H_kv=2, b=64, len_lo=300, len_hi=5000, B=3, n_local=2, paged=True), 128),  # 3 blocks touched
     (dict(H_q=8, H_kv=2, b=128, len_lo=1000, len_hi=4000, B=2, n_local=2), 64),     # window inside a block
     (dict(H_q=4, H_kv=1, b=64, len_lo=64, len_hi=64, n_local=1), 64),               # every token new
+    (dict(H_q=8, H_kv=2, b=128, len_lo=1000, len_hi=1000, n_local=2), 128),         # 128 tokens over 2 blocks
+    (dict(H_q=32, H_kv=2, b=64, len_lo=3000, len_hi=3000, n_local=2), 16),          # 256 rows: 2 row groups
 ]
 
 
