@@ -126,6 +126,15 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def bf16_peak():
+    """Dense bf16 tensor throughput (TFLOP/s) of one B200 for a kernel timed as a burst."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 # sources of the fused step kernel: a recorded ncu traffic figure is valid only while they are unchanged
 KERNEL_SOURCES = {
     "decode_step": ["fused_step.cu", "decode_tile.cuh", "select.cuh", "common.cuh", "launch.cuh"],
@@ -373,6 +382,24 @@ def rect_bytes(w, lens):
     return tot
 
 
+def rect_flops(w, lens, rows_per_cta=128):
+    """Tensor-core work of one rectification pass of one layer: (algorithmic, executed) flops.
+    Algorithmic: Q K^T and P V of every query row over the tokens it sees (row i of the window
+    sees L - f + i + 1).  Executed: every 64-token stage against every 128-row tile, with P V
+    issued twice (P's bf16 hi and lo parts)."""
+    f, G, d = w.rectify_every, w.H_q // w.H_kv, w.d
+    tiles = -(-f * G // rows_per_cta)
+    alg = ex = 0
+    for L in lens:
+        L = int(L)
+        if L <= 0:
+            continue
+        seen = sum(L - f + i + 1 for i in range(f))
+        alg += 4 * d * G * seen * w.H_kv
+        ex += 2 * d * rows_per_cta * tiles * (-(-L // 64) * 64) * 3 * w.H_kv
+    return alg, ex
+
+
 def native(args, rank, world, local, w=None, sweep=False):
     import torch
 
@@ -422,11 +449,18 @@ def native(args, rank, world, local, w=None, sweep=False):
         r_ms = max_over_ranks(r_ms, world, dev)
         rb = rect_bytes(w, lens) * n_layers
         hbm, _ = peaks()
+        tc, tc_src = bf16_peak()
+        fa, fe = (x * n_layers for x in rect_flops(w, lens))
         rect = {"every_steps": f, "us_per_pass": round(r_ms * 1e3, 1), "us_per_layer": round(r_ms * 1e3 / n_layers, 2),
                 "bytes_per_pass": rb, "gbs": round(job_gbs(rb, world, r_ms), 1),
                 "frac_of_measured_hbm": round(job_gbs(rb, 1, r_ms) / hbm, 4),
+                "tensor": {"flops_per_pass": fa, "executed_flops_per_pass": fe,
+                           "tflops": round(fa / (r_ms * 1e-3) / 1e12, 1),
+                           "executed_tflops": round(fe / (r_ms * 1e-3) / 1e12, 1),
+                           "peak": tc, "peak_source": tc_src,
+                           "frac_executed": round(fe / (r_ms * 1e-3) / 1e12 / tc, 4)},
                 "num_splits": S_r, "row_groups": rg,
-                "kernels": "mq_decode_kernel<dense> + combine_kernel per layer (one CUDA graph)"}
+                "kernels": "rect_tc_kernel (tcgen05) + combine_kernel per layer (one CUDA graph)"}
         del rgraph
 
     def step():

@@ -219,8 +219,7 @@ int sba_sparse_decode_multi(const sba_cache* c, const void* q, int32_t M, const 
     const int rc = check_multi(c, q, M, softmax_scale, num_splits, o_part, lse_part);
     if (rc != SBA_OK) return rc;
     if (!sel_idx || !sel_cnt || n_max < 1) return SBA_ERR_INVALID_ARG;
-    return after_launch(launch_multi_query(*c, q, M, sel_idx, sel_cnt, n_max, nullptr, nullptr, false,
-                                           softmax_scale, num_splits, o_part, lse_part,
+    return after_launch(launch_multi_query(*c, q, M, sel_idx, sel_cnt, n_max, softmax_scale, num_splits, o_part, lse_part,
                                            static_cast<cudaStream_t>(stream)));
 }
 

@@ -298,20 +298,27 @@ __device__ __forceinline__ void decode_block_t(DecodeStateT<NH>& st, const uint3
         }
         __syncwarp();
     }
-    // ---- S^T = K Q^T (16 tokens x 8 heads per n-tile) ----
-    float s[NH][4];
+    // ---- S^T = K Q^T (16 tokens x 8 heads per n-tile): two independent accumulator chains
+    // (even and odd channel steps), summed once ----
+    float s[NH][4], s2[NH][4];
 #pragma unroll
-    for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = 0.f;
+    for (int nh = 0; nh < NH; ++nh) s[nh][0] = s[nh][1] = s[nh][2] = s[nh][3] = s2[nh][0] = s2[nh][1] = s2[nh][2] = s2[nh][3] = 0.f;
     {
         const int row = tok0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        uint32_t a[8][4];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const int chunk = 2 * ks + (lane >> 4);
-            uint32_t a[4];
-            ldmatrix_x4(swz(kb + (chunk >> 3) * TG::kHalf, row, chunk & 7), a[0], a[1], a[2], a[3]);
-#pragma unroll
-            for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(s[nh], a, qb[nh][ks][0], qb[nh][ks][1]);
+            ldmatrix_x4(swz(kb + (chunk >> 3) * TG::kHalf, row, chunk & 7), a[ks][0], a[ks][1], a[ks][2], a[ks][3]);
         }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int nh = 0; nh < NH; ++nh) mma_bf16_16816((ks & 1) ? s2[nh] : s[nh], a[ks], qb[nh][ks][0], qb[nh][ks][1]);
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) s[nh][x] += s2[nh][x];
     }
     // ---- scale, log-gate, mask; online softmax over the tokens of each head (base 2) ----
     const int tr = lane >> 2;  // this lane's tokens: tr and tr + 8

@@ -695,15 +695,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                                 for (int x = 0; x < 4; ++x)
                                     acc[tl][nt][x][0] = acc[tl][nt][x][1] = acc[tl][nt][x][2] = acc[tl][nt][x][3] = 0.f;
+                        // every shared-memory read of the tile first, so that they are all in flight
+                        // together; the MMA chains then run on registers
+                        float4 xs[kTl][8][2];
 #pragma unroll
-                        for (int p = 0; p < 8; ++p) {
+                        for (int p = 0; p < 8; ++p)
 #pragma unroll
                             for (int tl = 0; tl < kTl; ++tl) {
                                 const int n0 = 16 * gw + 64 * (it0 + tl);
                                 const int R0 = (n0 + gq) * 4 + (p >> 1);
                                 const int off = ((((p & 1) << 2) | t) ^ (R0 & 7)) << 4;
-                                const float4 x0 = *reinterpret_cast<const float4*>(stage + R0 * 128 + off);
-                                const float4 x1 = *reinterpret_cast<const float4*>(stage + (R0 + 32) * 128 + off);
+                                xs[tl][p][0] = *reinterpret_cast<const float4*>(stage + R0 * 128 + off);
+                                xs[tl][p][1] = *reinterpret_cast<const float4*>(stage + (R0 + 32) * 128 + off);
+                            }
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+#pragma unroll
+                            for (int tl = 0; tl < kTl; ++tl) {
+                                const float4 x0 = xs[tl][p][0];
+                                const float4 x1 = xs[tl][p][1];
 #pragma unroll
                                 for (int e = 0; e < 2; ++e) {
                                     const float v[4] = {e ? x0.z : x0.x, e ? x1.z : x1.x, e ? x0.w : x0.y,

@@ -1,24 +1,16 @@
-// Several query tokens per sequence sharing one block selection, and the dense
-// causal rectification pass.
+// Several query tokens per sequence sharing one block selection.
 //
 // "Rectified Sparse Attention for Efficient Long-Sequence Generation",
-// Summary: after every f generated tokens those f tokens are re-encoded in one
-// parallel dense pass (their keys and values rewritten, the block keys of the
-// touched blocks refreshed); all query heads of a GQA group share one block
-// selection.  Key points: f in {16, 32, 64, 128}; ReSA is compared with
-// sparse-KV self-speculative decoding, which checks several draft tokens with
-// one sparse pass.
-//
-// Both are the same computation over different block lists: the M query
-// tokens of a sequence sit at its last M positions (len-M .. len-1), token i
-// attends causally to positions t <= len-M+i, and every one of the M*G query
-// rows of a (sequence, KV group) reads each staged K/V tile once:
-//  - sparse (sba_sparse_decode_multi): the group's selected blocks, ranked by
-//    the Quest score summed over the group's heads and the M tokens
-//    (sba_score_select_multi);
-//  - dense (sba_rectify): every block [0, N); the M tokens' keys and values
-//    are written into the cache first, and the Quest descriptors of the blocks
-//    they touch are recomputed from the staged tiles.
+// Summary and Key points: all query heads of a GQA group share one block
+// selection, and ReSA is compared with sparse-KV self-speculative decoding,
+// which checks several draft tokens with one sparse pass.  The M query tokens
+// of a sequence sit at its last M positions (len-M .. len-1), token i attends
+// causally to positions t <= len-M+i of the group's selected blocks (ranked by
+// the Quest score summed over the group's heads and the M tokens,
+// sba_score_select_multi), and every one of the M*G query rows of a
+// (sequence, KV group) reads each staged K/V tile once.  (The dense causal
+// pass over every block, the rectification, runs on the tcgen05 tensor cores
+// in rect_tc.cu.)
 //
 // One CTA per (split, KV head x row group, sequence).  A row group is up to
 // 128 query rows (row r of a group = token r / G, head r % G), i.e. 8 tiles of
@@ -59,11 +51,9 @@ struct MqArgs {
     sba_cache c;
     const __nv_bfloat16* q;  // [B][M][H_q][d]
     int M;
-    const int32_t* sel_idx;  // sparse: [B][H_kv][n_max]
-    const int32_t* sel_cnt;  // sparse: [B][H_kv]
+    const int32_t* sel_idx;  // [B][H_kv][n_max]
+    const int32_t* sel_cnt;  // [B][H_kv]
     int n_max;
-    const uint4* k_new;      // dense: [B][M][H_kv][d], the keys of positions len-M .. len-1
-    const uint4* v_new;
     float scale_log2;
     int num_splits;
     int row_groups;          // CTAs along the M*G query rows of a group
@@ -168,18 +158,7 @@ __device__ __forceinline__ void mq_chunk16(MqState& st, const uint32_t (&qa)[8][
     }
 }
 
-__device__ __forceinline__ uint32_t bf16x2_min2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint32_t bf16x2_max2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-template <int kBlk, bool kDense>
+template <int kBlk>
 __global__ void __launch_bounds__(kMqThreads, 1)
     mq_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ MqArgs a) {
@@ -226,25 +205,15 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         len = N * kBlk;
     }
     const int pos0 = len - a.M;  // first query token's position
-    // the block list: every block (dense) or the group's selection (sparse)
-    int cnt;
-    const int32_t* sel = nullptr;
-    if (kDense) {
-        cnt = N;
-    } else {
-        cnt = __ldg(a.sel_cnt + s * c.H_kv + h);
-        if (cnt > a.n_max || cnt < 0) {
-            if (tid == 0 && sp == 0 && rg == 0) report(c.status, SBA_DEV_BAD_SELECTION);
-            cnt = cnt < 0 ? 0 : a.n_max;
-        }
-        sel = a.sel_idx + ((int64_t)s * c.H_kv + h) * a.n_max;
+    // the group's selection
+    int cnt = __ldg(a.sel_cnt + s * c.H_kv + h);
+    if (cnt > a.n_max || cnt < 0) {
+        if (tid == 0 && sp == 0 && rg == 0) report(c.status, SBA_DEV_BAD_SELECTION);
+        cnt = cnt < 0 ? 0 : a.n_max;
     }
+    const int32_t* sel = a.sel_idx + ((int64_t)s * c.H_kv + h) * a.n_max;
     const int i0 = (int)((int64_t)cnt * sp / a.num_splits), i1 = (int)((int64_t)cnt * (sp + 1) / a.num_splits);
     const int nfill = (i1 - i0) * kSub;
-    // dense: blocks holding the M new tokens (written here, their descriptors refreshed)
-    const bool appends = kDense && a.M > 0 && pos0 >= 0;
-    if (kDense && pos0 < 0 && tid == 0 && sp == 0 && blockIdx.y == 0) report(c.status, SBA_DEV_BAD_POSITION);
-    const int tb0 = appends ? pos0 / kBlk : N;
 
     const bool consumer = warp < NCW && rows > 0;
     MqState stt;  // a consumer warp's 16 rows (registers), stored for the merge at the end
@@ -260,7 +229,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 alive = __shfl_sync(0xffffffffu, alive, 0);
                 if (!alive) break;
             }
-            int j = kDense ? i : __ldg(sel + i);
+            const int j = __ldg(sel + i);
             int pg = -1;
             if (j >= 0 && j < N) {
                 pg = (int)page_of(c, s, j, lane == 0 ? c.status : nullptr);
@@ -275,19 +244,6 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 }
                 __syncwarp();
                 continue;
-            }
-            if (appends && sb == 0 && j >= tb0) {
-                // the new tokens of this block: 2 x 16 16-byte pieces per token, then this lane's
-                // stores are ordered ahead of the tile loads below
-                const int t0 = max(pos0, j * kBlk), t1 = min(len, (j + 1) * kBlk);
-                for (int e = lane; e < (t1 - t0) * 32; e += 32) {
-                    const int t = t0 + (e >> 5), half = (e >> 4) & 1, l = e & 15;
-                    const int64_t src = (((int64_t)s * a.M + (t - pos0)) * c.H_kv + h) * 16 + l;
-                    const uint4 v = __ldg((half ? a.v_new : a.k_new) + src);
-                    reinterpret_cast<uint4*>(half ? c.v : c.k)[(((int64_t)pg * c.H_kv + h) * kBlk + t % kBlk) * 16 + l] = v;
-                }
-                fence_proxy_async_global();
-                __syncwarp();
             }
             if (lane == 0) {
                 info[st] = MqStage{j, sb, valid, 1};
@@ -318,52 +274,6 @@ __global__ void __launch_bounds__(kMqThreads, 1)
                 if (!ok) alive = false;
             }
             __syncwarp();
-        }
-        // dense: the Quest descriptors of the blocks the new tokens touched, from their staged K
-        // rows (the last fills of this share, still in the ring: nothing is loaded after them)
-        if (appends && c.desc && rg == 0 && alive) {
-            for (int f = max(0, nfill - kMqStages); f < nfill; ++f) {
-                const int i = i0 + f / kSub, sb = f % kSub;
-                if (sb != 0 || i < tb0) continue;
-                const int j = i;
-                const int vb = min(kBlk, len - j * kBlk);  // the block's valid tokens
-                if (vb <= 0 || f + (vb > 64 ? 1 : 0) >= nfill) continue;
-                uint32_t mn[4], mx[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) mn[e] = 0x7f807f80u, mx[e] = 0xff80ff80u;
-                bool ok = true;
-                for (int sub = 0; sub < kSub && ok; ++sub) {
-                    const int ff = f + sub, vs = min(64, vb - 64 * sub);
-                    if (vs <= 0) break;
-                    if (lane == 0) ok = mbar_wait(&full[ff % kMqStages], (ff / kMqStages) & 1, c.status);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    const uint8_t* kt = dyn + (size_t)(ff % kMqStages) * kMqStage;
-                    const int ck = lane & 15, cc = ck & 7;
-                    for (int t = lane >> 4; t < vs; t += 2) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(kt + (ck >> 3) * kMqHalf + t * 128 +
-                                                                          ((cc ^ (t & 7)) << 4));
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            mn[e] = bf16x2_min2(mn[e], ws[e]);
-                            mx[e] = bf16x2_max2(mx[e], ws[e]);
-                        }
-                    }
-                }
-                if (!ok) break;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    mn[e] = bf16x2_min2(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], 16));
-                    mx[e] = bf16x2_max2(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
-                }
-                const int pg = (int)page_of(c, s, j, nullptr);
-                if (lane < 16 && pg >= 0) {
-                    uint8_t* d = reinterpret_cast<uint8_t*>(c.desc) + ((int64_t)pg * c.H_kv + h) * 2 * kHeadDim * 2;
-                    *reinterpret_cast<uint4*>(d + lane * 16) = make_uint4(mn[0], mn[1], mn[2], mn[3]);
-                    *reinterpret_cast<uint4*>(d + 2 * kHeadDim + lane * 16) = make_uint4(mx[0], mx[1], mx[2], mx[3]);
-                }
-            }
         }
     } else if (consumer) {
         // ------------------------------ consumers -----------------------------
@@ -429,7 +339,7 @@ __global__ void __launch_bounds__(kMqThreads, 1)
         stt.l1 += __shfl_xor_sync(0xffffffffu, stt.l1, 1);
         stt.l1 += __shfl_xor_sync(0xffffffffu, stt.l1, 2);
     }
-    __syncthreads();  // every consumer and the producer (its refresh included) are done with the ring
+    __syncthreads();  // every consumer and the producer are done with the ring
     if (consumer) {
         // this warp's rows to shared memory (the ring) for the token-slot merge
         float* mo = reinterpret_cast<float*>(dyn) + warp * 16 * kHeadDim;
@@ -470,14 +380,14 @@ __global__ void __launch_bounds__(kMqThreads, 1)
     }
 }
 
-template <int kBlk, bool kDense>
+template <int kBlk>
 int launch_mq_t(const sba_cache& c, const MqArgs& a, cudaStream_t stream) {
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
     if (!make_kv_tmap(&tk, c.k, rows, 64) || !make_kv_tmap(&tv, c.v, rows, 64)) return SBA_ERR_CUDA;
-    if (allow_smem<mq_decode_kernel<kBlk, kDense>>(kMqSmem) != SBA_OK) return SBA_ERR_CUDA;
+    if (allow_smem<mq_decode_kernel<kBlk>>(kMqSmem) != SBA_OK) return SBA_ERR_CUDA;
     dim3 grid(a.num_splits, c.H_kv * a.row_groups, c.B);
-    return launch(mq_decode_kernel<kBlk, kDense>, grid, dim3(kMqThreads), kMqSmem, stream, tk, tv, a);
+    return launch(mq_decode_kernel<kBlk>, grid, dim3(kMqThreads), kMqSmem, stream, tk, tv, a);
 }
 
 }  // namespace
@@ -488,7 +398,7 @@ int mq_row_groups(const sba_cache& c, int M) {
 }
 
 int launch_multi_query(const sba_cache& c, const void* q, int M, const int32_t* sel_idx, const int32_t* sel_cnt,
-                       int n_max, const void* k_new, const void* v_new, bool dense, float scale, int num_splits,
+                       int n_max, float scale, int num_splits,
                        float* o_part, float* lse_part, cudaStream_t stream) {
     MqArgs a{};
     a.c = c;
@@ -497,15 +407,12 @@ int launch_multi_query(const sba_cache& c, const void* q, int M, const int32_t* 
     a.sel_idx = sel_idx;
     a.sel_cnt = sel_cnt;
     a.n_max = n_max;
-    a.k_new = reinterpret_cast<const uint4*>(k_new);
-    a.v_new = reinterpret_cast<const uint4*>(v_new);
     a.scale_log2 = scale * kLog2e;
     a.num_splits = num_splits;
     a.row_groups = mq_row_groups(c, M);
     a.o_part = o_part;
     a.lse_part = lse_part;
-    if (dense) return c.b == 64 ? launch_mq_t<64, true>(c, a, stream) : launch_mq_t<128, true>(c, a, stream);
-    return c.b == 64 ? launch_mq_t<64, false>(c, a, stream) : launch_mq_t<128, false>(c, a, stream);
+    return c.b == 64 ? launch_mq_t<64>(c, a, stream) : launch_mq_t<128>(c, a, stream);
 }
 
 }  // namespace sba
