@@ -156,6 +156,9 @@ int sba_score_select(const sba_cache* c, const void* q, const sba_select_params*
                                             n_max, ws, static_cast<cudaStream_t>(stream)));
 }
 
+// a softmax scale is positive and finite
+static bool good_scale(float s) { return s > 0.f && s <= 3.4028234e38f; }
+
 static int sparse_decode_any(const sba_cache* c, const void* q, const int32_t* sel_idx, const int32_t* sel_cnt,
                              const float* gate_bias, int32_t n_max, float softmax_scale, int32_t num_splits,
                              float* o_part, float* lse_part, bool outer, void* stream) {
@@ -164,7 +167,7 @@ static int sparse_decode_any(const sba_cache* c, const void* q, const int32_t* s
     if (!q || !sel_idx || !sel_cnt || !o_part || !lse_part || n_max < 1) return SBA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(o_part)) return SBA_ERR_INVALID_ARG;
     if (num_splits < 1 || num_splits > 65535) return SBA_ERR_INVALID_ARG;
-    if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return SBA_ERR_INVALID_ARG;
+    if (!good_scale(softmax_scale)) return SBA_ERR_INVALID_ARG;
     if (outer && !gate_bias) return SBA_ERR_INVALID_ARG;
     return after_launch(launch_sparse_decode(*c, q, sel_idx, sel_cnt, gate_bias, n_max, softmax_scale, num_splits,
                                              o_part, lse_part, outer, static_cast<cudaStream_t>(stream)));
@@ -203,7 +206,7 @@ static int check_multi(const sba_cache* c, const void* q, int32_t M, float softm
     if (!q || !o_part || !lse_part || !aligned16(q)) return SBA_ERR_INVALID_ARG;
     if (M < 1 || M > kMaxQueryTokens) return SBA_ERR_INVALID_ARG;
     if (num_splits < 1 || num_splits > 65535) return SBA_ERR_INVALID_ARG;
-    if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return SBA_ERR_INVALID_ARG;
+    if (!good_scale(softmax_scale)) return SBA_ERR_INVALID_ARG;
     if ((int64_t)c->H_kv * mq_row_groups(*c, M) > 65535 || c->B > 65535) return SBA_ERR_UNSUPPORTED;
     return SBA_OK;
 }
@@ -266,7 +269,7 @@ int sba_decode_step(const sba_cache* c, const void* q, const void* k_new, const 
     if (rc != SBA_OK) return rc;
     if (!q || !out || !aligned16(q) || n_new < 0) return SBA_ERR_INVALID_ARG;
     if (out_dtype != SBA_OUT_F32 && out_dtype != SBA_OUT_BF16) return SBA_ERR_INVALID_ARG;
-    if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return SBA_ERR_INVALID_ARG;
+    if (!good_scale(softmax_scale)) return SBA_ERR_INVALID_ARG;
     if (n_new > 0 && (!k_new || !v_new || !pos_start || !aligned16(k_new) || !aligned16(v_new)))
         return SBA_ERR_INVALID_ARG;
     if (p->scorer == SBA_SCORER_QUEST && !c->desc) return SBA_ERR_INVALID_ARG;

@@ -13,7 +13,7 @@ constexpr int kHeadDim = 128;
 constexpr int kMaxGroup = 16;
 constexpr int kMaxBlocksPerSeq = 32768;  // selection keys live in shared memory
 constexpr int kMaxQueryTokens = 1024;   // query tokens per sequence of the multi-token calls
-constexpr int kMaxRectifyTokens = 128;  // rectification window: its blocks stay in the staging ring
+constexpr int kMaxRectifyTokens = 128;  // rectification window: the pages' largest f
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bounded waits give up after ~2 s
 
 // ---------------------------------------------------------------------------
@@ -145,6 +145,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            report(status, SBA_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// The same wait, each try suspending the thread until the phase completes or about
+// `hint_ns` pass: a waiting warp then takes no issue slots from the working ones.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, int32_t* status,
+                                                uint32_t hint_ns = 20000) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_hint(bar, parity, hint_ns)) {
         if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
             report(status, SBA_DEV_TIMEOUT);
             return false;

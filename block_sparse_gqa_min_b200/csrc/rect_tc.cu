@@ -8,34 +8,41 @@
 // key and value tile, this is a dense contraction: 128 query rows against each
 // 64-token tile, the shape the tensor cores take whole.
 //
-// One CTA per (split, KV head x row group of 128 query rows, sequence); 320
+// One CTA per (split, KV head x row group of 128 query rows, sequence); 576
 // threads:
-//  - warp 8 (producer) streams each block in 64-token stages (K0 K1 V0 V1: four
+//  - warp 16 (producer) streams each block in 64-token stages (K0 K1 V0 V1: four
 //    2-D TMA loads of 64 rows x 128 B, 128-byte swizzle, no multicast) into a
-//    ring of 32 KB stages.  Before a block the window touches is loaded, it
+//    ring of six 32 KB stages (shared memory holds nothing else: Q and P live in
+//    TMEM).  Before a block the window touches is loaded, it
 //    writes the window's K/V rows of that block into the cache (a proxy fence
 //    orders them ahead of the tile load); after its last fill it recomputes the
 //    Quest min/max of those blocks from their keys.  Rows past len are zeroed in
 //    the stage before anyone reads it.
-//  - warp 9 (MMA) allocates 256 TMEM columns and, one thread issuing, runs
+//  - warp 17 (MMA) allocates all 512 TMEM columns and, one thread issuing, runs
 //    S = Q K^T for each stage (M 128 rows, N 64 tokens, K 128 channels: eight
-//    tcgen05.mma kind::f16, bf16 in, fp32 accumulate) into one of two TMEM S
-//    buffers (columns 0-63, 64-127), so the next stage's S is computed while
-//    the softmax works on this one; then, once P is written,
-//    O += P_hi V + P_lo V (M 128, N 128 channels, K 64 tokens; V read MN-major
-//    straight from the TMA tile) into TMEM columns 128-255.  tcgen05.commit
-//    signals S, O and the stage's release on mbarriers.
-//  - warps 0-7 (softmax): query row r = TMEM lane r is shared by warps r/32
-//    and r/32 + 4, each owning 32 of the stage's 64 columns.  A thread reads
-//    its half row of S (tcgen05.ld 32x32b.x32), applies the causal limit
-//    (t <= len - f + i for token i) and the scale, agrees on the row maximum
-//    with its partner through shared memory, keeps an online softmax whose
-//    exponent offset moves only when the row maximum grows by more than 2^8
-//    (then O's row is rescaled in TMEM; otherwise exponentials stay below
-//    2^8), and writes its half of P as bf16 hi + lo parts (about 16 mantissa
-//    bits) into one of two 128-byte-swizzled A tiles.  At the end it reads its
-//    64 columns of O, normalises them and writes the split's O and LSE
-//    ([B][f][H_q][S][d], [B][f][H_q][S]).
+//    tcgen05.mma kind::f16, bf16 in, fp32 accumulate; A = Q from TMEM, B = the
+//    K tile) into one of two TMEM S buffers (columns 0-63, 64-127), so the next
+//    stage's S is computed while the softmax works on this one; then, once P
+//    is written, O += P_hi V + P_lo V (M 128, N 128 channels, K 64 tokens;
+//    A = P from TMEM, V read MN-major straight from the TMA tile) into TMEM
+//    columns 128-255.  tcgen05.commit signals S, O and the stage's release on
+//    mbarriers.  A 16-bit A operand in TMEM is row r = lane r with two
+//    consecutive K elements per 32-bit column (the lower one in the low half):
+//    Q takes columns 384-447 (128 channels), each of the two P buffers 64
+//    columns from 256 (32 for the hi parts of its 64 tokens, then 32 for the lo).
+//  - warps 0-15 (softmax): query row r = TMEM lane r is shared by the four
+//    warps w with w % 4 = r / 32, warp w owning columns 16 (w / 4) .. + 15 of
+//    each 64-token stage.  A thread reads its 16 columns of S (tcgen05.ld
+//    32x32b.x16), applies the causal limit (t <= len - f + i for token i),
+//    agrees on the row maximum with the other three warps through shared
+//    memory, keeps an online softmax in base 2 (the scale folded into the
+//    exponent's FMA) whose offset moves only when the row maximum grows by
+//    more than 2^8 (then O's row is rescaled in TMEM; otherwise exponentials
+//    stay below 2^8), and writes its 16 tokens of P as bf16 hi + lo parts
+//    (hi + lo within 2^-15 |p| of p) into one of the two TMEM P buffers
+//    (tcgen05.st).
+//    At the end it reads its 32 columns of O, normalises them and writes the
+//    split's O and LSE ([B][f][H_q][S][d], [B][f][H_q][S]).
 // Every wait is bounded: a wait that runs out reports SBA_DEV_TIMEOUT and the
 // roles stop, and TMEM is released on every path.
 #include <cuda.h>
@@ -50,20 +57,28 @@ namespace sba {
 
 bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);  // decode.cu
 
+#ifndef SBA_RECT_SOFTMAX_WARPS
+#define SBA_RECT_SOFTMAX_WARPS 8
+#endif
+
 namespace {
 
 constexpr int kRtRows = 128;               // query rows per CTA: the MMA's M
-constexpr int kRtStages = 3;               // 64-token K/V stages (with the two P buffers, all that fits)
+constexpr int kRtStages = 6;               // 64-token K/V stages: 192 KB, all the shared memory there is
 constexpr int kRtStage = 32768;
 constexpr int kRtHalf = 8192;              // 64 rows x 128 B
-constexpr int kRtThreads = 320;            // warps 0-7 softmax, 8 producer, 9 MMA
-constexpr int kProdWarp = 8, kMmaWarp = 9;
-constexpr int kOffQ = 0;                   // 2 x 16 KB: 128 rows x 64 channels, K-major, 128-B swizzle
-constexpr int kOffP = 32768;               // two P buffers of 32 KB: hi (16 KB) then lo, 128 rows x 64 tokens
-constexpr int kOffRing = 98304;
-constexpr int kRtSmem = kOffRing + kRtStages * kRtStage + 1024;
-constexpr uint32_t kTmemCols = 256;        // S buffers: columns 0-63 and 64-127; O: 128-255
-constexpr uint32_t kColS = 0, kColO = 128;
+constexpr int kSmWarps = SBA_RECT_SOFTMAX_WARPS;  // softmax warps: kCq per TMEM lane quarter
+constexpr int kCq = kSmWarps / 4;          // warps sharing a query row (column groups)
+constexpr int kCols = 64 / kCq;            // S columns (tokens) of a stage per thread
+constexpr int kOCols = 128 / kCq;          // O (and Q) channels per thread
+constexpr int kRtThreads = (kSmWarps + 2) * 32;  // softmax warps, then the producer, then the MMA warp
+constexpr int kProdWarp = kSmWarps, kMmaWarp = kSmWarps + 1;
+static_assert(kSmWarps == 8 || kSmWarps == 16, "two or four warps per TMEM lane quarter");
+constexpr int kRtSmem = kRtStages * kRtStage + 1024;
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns: S buffers 0-63 and 64-127 (fp32); O 128-255 (fp32); P buffers 256-319 and
+// 320-383 (bf16 pairs: hi parts in the first 32, lo parts in the next 32); Q 384-447 (bf16 pairs)
+constexpr uint32_t kColS = 0, kColO = 128, kColP = 256, kColQ = 384;
 
 struct RtArgs {
     sba_cache c;
@@ -89,11 +104,13 @@ __host__ __device__ constexpr uint32_t umma_idesc(int M, int N, bool b_mn_major)
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// D (+)= A B with A read from TMEM (K-major: row = lane, two 16-bit K elements per column) and B
+// from shared memory
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc));
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -102,26 +119,7 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 64 consecutive TMEM columns of this thread's lane (warp w reads lanes 32w..32w+31).
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-    uint32_t r[64];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,"
-        "%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
-}
+// consecutive TMEM columns of this thread's lane (warp w accesses lanes 32 (w % 4) ..)
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
     asm volatile(
@@ -136,6 +134,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 // 2^x by the special-function unit (flushes results below 2^-126 to zero, which no softmax
 // weight here can reach with any effect)
 __device__ __forceinline__ float ex2(float x) {
@@ -145,35 +154,54 @@ __device__ __forceinline__ float ex2(float x) {
 }
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
+// 8 / 16 / 32 consecutive 32-bit TMEM columns of this thread's lane, from registers; the caller
+// waits (tcgen05.wait::st) before signalling
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,"
-        "%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
             taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31])), "r"(__float_as_uint(v[32])),
-        "r"(__float_as_uint(v[33])), "r"(__float_as_uint(v[34])), "r"(__float_as_uint(v[35])),
-        "r"(__float_as_uint(v[36])), "r"(__float_as_uint(v[37])), "r"(__float_as_uint(v[38])),
-        "r"(__float_as_uint(v[39])), "r"(__float_as_uint(v[40])), "r"(__float_as_uint(v[41])),
-        "r"(__float_as_uint(v[42])), "r"(__float_as_uint(v[43])), "r"(__float_as_uint(v[44])),
-        "r"(__float_as_uint(v[45])), "r"(__float_as_uint(v[46])), "r"(__float_as_uint(v[47])),
-        "r"(__float_as_uint(v[48])), "r"(__float_as_uint(v[49])), "r"(__float_as_uint(v[50])),
-        "r"(__float_as_uint(v[51])), "r"(__float_as_uint(v[52])), "r"(__float_as_uint(v[53])),
-        "r"(__float_as_uint(v[54])), "r"(__float_as_uint(v[55])), "r"(__float_as_uint(v[56])),
-        "r"(__float_as_uint(v[57])), "r"(__float_as_uint(v[58])), "r"(__float_as_uint(v[59])),
-        "r"(__float_as_uint(v[60])), "r"(__float_as_uint(v[61])), "r"(__float_as_uint(v[62])),
-        "r"(__float_as_uint(v[63]))
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// N consecutive fp32 columns (N = 16, 32 or 64) into / from registers
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(v));
+    } else {
+        static_assert(N % 32 == 0, "");
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i) tmem_ld32(taddr + 32 * i, *reinterpret_cast<float(*)[32]>(v + 32 * i));
+    }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* v) {
+    if constexpr (N == 8) {
+        tmem_st8(taddr, *reinterpret_cast<const uint32_t(*)[8]>(v));
+    } else if constexpr (N == 16) {
+        tmem_st16(taddr, *reinterpret_cast<const uint32_t(*)[16]>(v));
+    } else {
+        static_assert(N % 32 == 0, "");
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i) tmem_st32(taddr + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(v + 32 * i));
+    }
 }
 
 __device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
@@ -194,10 +222,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     constexpr int kSub = kBlk / 64;
     extern __shared__ uint8_t dyn_raw[];
     uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t kv_full[kRtStages], kv_empty[kRtStages], zbar, s_full[2], p_full[2], pv_done[2], fin;
+    __shared__ uint64_t kv_full[kRtStages], kv_empty[kRtStages], zbar, q_full, s_full[2], p_full[2], pv_done[2], fin;
     __shared__ uint32_t tmem_base;
-    __shared__ float xmax[2][2][kRtRows];  // [stage parity][column half][row]: partial row maxima
-    __shared__ float xl[2][kRtRows];       // [column half][row]: partial row sums at the end
+    __shared__ float xmax[2][kCq][kRtRows];  // [stage parity][column group][row]: partial row maxima
+    __shared__ float xl[kCq][kRtRows];       // [column group][row]: partial row sums at the end
 
     const sba_cache& c = a.c;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -212,9 +240,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             mbar_init(&kv_empty[i], 1);
         }
         mbar_init(&zbar, 1);
+        mbar_init(&q_full, kSmWarps);  // one arrival per softmax warp
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 8);  // one arrival per softmax warp
+            mbar_init(&p_full[b], kSmWarps);
             mbar_init(&pv_done[b], 1);
         }
         mbar_init(&fin, 1);
@@ -253,22 +282,31 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     // processed fills are fills 0 .. nproc-1 for every role
     const int nproc = (nfill > 0 && fill_valid(nfill - 1) == 0) ? nfill - 1 : nfill;
 
-    // the query rows of this CTA into the K-major, 128-byte-swizzled A tile (zero past the group's rows)
-    if (warp < 8) {
-        const int r = tid & 127, half = tid >> 7, gr = row0 + r;
+    // this thread's share of its query row (row = TMEM lane 32 (warp % 4) + lane, channels
+    // kOCols (warp / 4) ..): zero past the group's rows
+    uint32_t qv[kOCols / 2];
+    if (warp < kSmWarps) {
+        const int r = 32 * (warp & 3) + lane, cq = warp >> 2, gr = row0 + r;
         const __nv_bfloat16* qrow =
             gr < R ? a.q + (((int64_t)s * a.M + gr / G) * c.H_q + h * G + gr % G) * kHeadDim : nullptr;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            const uint4 v = qrow ? __ldg(reinterpret_cast<const uint4*>(qrow) + 8 * half + cc) : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(dyn + kOffQ + half * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+        for (int cc = 0; cc < kOCols / 8; ++cc) {
+            const uint4 v = qrow ? __ldg(reinterpret_cast<const uint4*>(qrow) + (kOCols / 8) * cq + cc)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+            qv[4 * cc] = v.x, qv[4 * cc + 1] = v.y, qv[4 * cc + 2] = v.z, qv[4 * cc + 3] = v.w;
         }
-        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = tmem_base;
+    if (warp < kSmWarps) {  // Q into its TMEM columns, then the MMA warp may read it
+        tmem_st_n<kOCols / 2>(tm + ((uint32_t)(32 * (warp & 3)) << 16) + kColQ + (kOCols / 2) * (warp >> 2), qv);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_full);
+    }
 
     bool alive = true;
     if (warp == kProdWarp) {
@@ -279,12 +317,12 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             const int i = i0 + q / kSub, sb = q % kSub, j = i;
             const int st = q % kRtStages;
             if (q >= kRtStages) {
-                if (lane == 0) alive = mbar_wait(&kv_empty[st], ((q / kRtStages) - 1) & 1, c.status);
+                if (lane == 0) alive = mbar_wait_sleep(&kv_empty[st], ((q / kRtStages) - 1) & 1, c.status);
                 alive = __shfl_sync(0xffffffffu, alive, 0);
                 if (!alive) break;
             }
             const int pg = (int)page_of(c, s, j, lane == 0 ? c.status : nullptr);
-            uint8_t* base = dyn + kOffRing + (size_t)st * kRtStage;
+            uint8_t* base = dyn + (size_t)st * kRtStage;
             if (pg < 0) {
                 // a bad table entry (reported): the stage is zeros, the roles stay in step
                 for (int e = lane; e < kRtStage / 16; e += 32) reinterpret_cast<uint4*>(base)[e] = make_uint4(0u, 0u, 0u, 0u);
@@ -370,28 +408,35 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // ------------------------------ MMA issue ------------------------------
         constexpr uint32_t kIdQK = umma_idesc(128, 64, false);
         constexpr uint32_t kIdPV = umma_idesc(128, 128, true);
-        const uint32_t sQ = smem_u32(dyn + kOffQ), sP0 = smem_u32(dyn + kOffP);
+        // descriptors of ring stage 0 (K tile: K-major; V tile: MN-major, its two 64-channel halves
+        // 8 KB apart); a stage or a K step adds its byte offset / 16 to the start-address field,
+        // which stays below 2^14 for every shared-memory address
+        const uint32_t ring = smem_u32(dyn);
+        const uint64_t dK0 = umma_desc(ring, 16, 1024), dV0 = umma_desc(ring + 2 * kRtHalf, kRtHalf, 1024);
         bool issued = false;  // any MMA issued by this warp
+        if (lane == 0) alive = mbar_wait_sleep(&q_full, 0, c.status);  // Q in TMEM
+        alive = __shfl_sync(0xffffffffu, alive, 0);
         // S(q) = Q K(q)^T into S buffer q % 2; K = 128 channels in eight steps of 16 (32 bytes
         // along the swizzled rows)
         auto issue_qk = [&](int q) {
             const int st = q % kRtStages;
-            if (lane == 0) alive = mbar_wait(&kv_full[st], (q / kRtStages) & 1, c.status);
+            if (lane == 0) alive = mbar_wait_sleep(&kv_full[st], (q / kRtStages) & 1, c.status);
             alive = __shfl_sync(0xffffffffu, alive, 0);
             if (!alive) return;
             tc_fence_after();
-            const uint32_t sK = smem_u32(dyn + kOffRing + (size_t)st * kRtStage);
+            const uint64_t dK = dK0 + (uint64_t)((st * kRtStage) >> 4);
+            const uint32_t tS = tm + kColS + 64 * (q & 1);
             if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tm + kColS + 64 * (q & 1), umma_desc(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                             umma_desc(sK + (kk >> 2) * kRtHalf + (kk & 3) * 32, 16, 1024), kIdQK, kk > 0);
+                    umma_f16_ts(tS, tm + kColQ + 8 * kk, dK + (uint64_t)((((kk >> 2) * kRtHalf) + (kk & 3) * 32) >> 4),
+                                kIdQK, kk > 0);
                 umma_commit(&s_full[q & 1]);
             }
             issued = true;
             __syncwarp();
         };
-        if (nproc > 0) issue_qk(0);
+        if (nproc > 0 && alive) issue_qk(0);
         for (int q = 0; q < nproc && alive; ++q) {
             // the next stage's S overlaps this stage's softmax (its S buffer was read by the softmax of
             // stage q - 1, whose P has been waited for)
@@ -399,22 +444,21 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 issue_qk(q + 1);
                 if (!alive) break;
             }
-            if (lane == 0) alive = mbar_wait(&p_full[q & 1], (q >> 1) & 1, c.status);
+            if (lane == 0) alive = mbar_wait_sleep(&p_full[q & 1], (q >> 1) & 1, c.status);
             alive = __shfl_sync(0xffffffffu, alive, 0);
             if (!alive) break;
             tc_fence_after();
             const int st = q % kRtStages;
-            const uint32_t sV = smem_u32(dyn + kOffRing + (size_t)st * kRtStage) + 2 * kRtHalf;
-            const uint32_t sP = sP0 + (q & 1) * 32768;
+            const uint64_t dV = dV0 + (uint64_t)((st * kRtStage) >> 4);
+            const uint32_t tP = tm + kColP + 64 * (q & 1);
             if (lane == 0) {
-                // O += P V: K = 64 tokens in four steps of 16 (two 8-row groups of the V tile each); V is
-                // MN-major, its two 64-channel halves 8 KB apart
+                // O += P V: K = 64 tokens in four steps of 16 (two 8-token groups of the V tile, 2 KB)
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tm + kColO, umma_desc(sP + part * 16384 + kk * 32, 16, 1024),
-                                 umma_desc(sV + kk * 2048, kRtHalf, 1024), kIdPV, (q > 0 || part > 0 || kk > 0));
+                        umma_f16_ts(tm + kColO, tP + 32 * part + 8 * kk, dV + (uint64_t)((kk * 2048) >> 4), kIdPV,
+                                    (q > 0 || part > 0 || kk > 0));
                 umma_commit(&pv_done[q & 1]);
                 umma_commit(&kv_empty[st]);
             }
@@ -429,47 +473,49 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------ softmax ------------------------------
-        const int qd = warp & 3, hf = warp >> 2;  // lane quarter, column half
+        const int qd = warp & 3, cq = warp >> 2;  // lane quarter, column group
         const int r = 32 * qd + lane;              // query row = TMEM lane
         const int gr = row0 + r;
         const int lim = gr < R ? pos0 + gr / G + 1 : 0;  // causal limit (exclusive)
         const uint32_t lane_base = tm + ((uint32_t)(qd * 32) << 16);
+        const float sl2 = a.scale_log2;
+        // m_used: the exponent offset in scaled base-2 units (-inf until the row has a valid token)
         float m_used = -INFINITY, l = 0.f;
         // (a wait that runs out turns this warp dead; a dead warp still takes every named barrier of the
-        // loop, so its partner never waits on it forever, and arrives on nothing)
+        // loop, so the row's other warps never wait on it forever, and arrives on nothing)
         for (int q = 0; q < nproc; ++q) {
             const int vf = fill_valid(q);
             const int j = i0 + q / kSub, sb = q % kSub;
-            const int base = j * kBlk + 64 * sb + 32 * hf;  // position of this half's first token
+            const int base = j * kBlk + 64 * sb + kCols * cq;  // position of this group's first token
             bool ok = alive;
             if (ok) {
-                if (lane == 0) ok = mbar_wait(&s_full[q & 1], (q >> 1) & 1, c.status);
+                if (lane == 0) ok = mbar_wait_sleep(&s_full[q & 1], (q >> 1) & 1, c.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
             }
-            float sv[32];
+            float sv[kCols];
             float mx = -INFINITY;
             if (ok) {
                 tc_fence_after();
-                tmem_ld32(lane_base + kColS + 64 * (q & 1) + 32 * hf, sv);
-                const int nval = min(32, min(vf - 32 * hf, lim - base));  // valid columns of this half row
-                if (nval >= 32) {
+                tmem_ld_n<kCols>(lane_base + kColS + 64 * (q & 1) + kCols * cq, sv);
+                const int nval = min(kCols, min(vf - kCols * cq, lim - base));  // valid columns of this group
+                if (nval < kCols) {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) sv[t] *= a.scale_log2;
-                } else {
-#pragma unroll
-                    for (int t = 0; t < 32; ++t) sv[t] = t < nval ? sv[t] * a.scale_log2 : -INFINITY;
+                    for (int t = 0; t < kCols; ++t) sv[t] = t < nval ? sv[t] : -INFINITY;
                 }
-                float m8[8];
+                float m4[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) m8[u] = fmaxf(fmaxf(sv[u], sv[u + 8]), fmaxf(sv[u + 16], sv[u + 24]));
+                for (int u = 0; u < 4; ++u) {
+                    m4[u] = sv[u];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) m8[u] = fmaxf(m8[u], m8[u + 4]);
-                mx = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+                    for (int t = u + 4; t < kCols; t += 4) m4[u] = fmaxf(m4[u], sv[t]);
+                }
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;  // the scale is positive
             }
-            // the row maximum agreed with the partner warp (the other half of the row's columns)
-            xmax[q & 1][hf][r] = mx;
-            named_bar(1 + qd, 64);
-            mx = fmaxf(mx, xmax[q & 1][hf ^ 1][r]);
+            // the row maximum agreed with the row's other warps
+            xmax[q & 1][cq][r] = mx;
+            named_bar(1 + qd, 32 * kCq);
+#pragma unroll
+            for (int x = 0; x < kCq; ++x) mx = fmaxf(mx, xmax[q & 1][x][r]);
             if (!ok) {
                 alive = false;
                 continue;
@@ -482,24 +528,32 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 l *= alpha;
             }
             const bool rescale = q > 0 && alpha != 1.f;
-            uint32_t ph[16], pl[16];
+            // (a row still without a valid token has every score at -inf: offset 0 gives 0 for each)
+            const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+            // P = hi + lo in bf16 by integer operations (no conversion instructions): hi = p with its
+            // low 16 bits cleared (truncation), r = p - hi (exact in fp32, 0 <= r < 2^-7 p) rounded to
+            // bf16 for lo by adding half a bf16 unit before its low 16 bits are dropped; the pair's
+            // upper halves are packed by one byte permute.  |p - hi - lo| <= 2^-8 r < 2^-15 p while r
+            // is a normal float (p >= 2^-100); below that the error is under 2^-130, nothing next to
+            // a row sum >= 1.
+            uint32_t ph[kCols / 2], pl[kCols / 2];
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int t = 0; t < 32; t += 2) {
-                const float p0 = m_used == -INFINITY ? 0.f : ex2(sv[t] - m_used);
-                const float p1 = m_used == -INFINITY ? 0.f : ex2(sv[t + 1] - m_used);
+            for (int t = 0; t < kCols; t += 2) {
+                const float p0 = ex2(fmaf(sv[t], sl2, neg_m));
+                const float p1 = ex2(fmaf(sv[t + 1], sl2, neg_m));
                 ls[(t >> 1) & 3] += p0 + p1;
-                const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-                const float2 hfv = __bfloat1622float2(hi);
-                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - hfv.x, p1 - hfv.y);
-                ph[t / 2] = *reinterpret_cast<const uint32_t*>(&hi);
-                pl[t / 2] = *reinterpret_cast<const uint32_t*>(&lo);
+                const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
+                const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                ph[t / 2] = __byte_perm(u0, u1, 0x7632);
+                pl[t / 2] = __byte_perm(__float_as_uint(r0) + 0x8000u, __float_as_uint(r1) + 0x8000u, 0x7632);
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             // this P buffer is free once O += P V of stage q - 2 has completed; O itself (to rescale)
             // once that of stage q - 1 has
             if (q >= 2) {
-                if (lane == 0) ok = mbar_wait(&pv_done[q & 1], ((q - 2) >> 1) & 1, c.status);
+                if (lane == 0) ok = mbar_wait_sleep(&pv_done[q & 1], ((q - 2) >> 1) & 1, c.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) {
                     alive = false;
@@ -508,37 +562,36 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 tc_fence_after();
             }
             if (__any_sync(0xffffffffu, rescale)) {
-                if (lane == 0) ok = mbar_wait(&pv_done[(q - 1) & 1], ((q - 1) >> 1) & 1, c.status);
+                if (lane == 0) ok = mbar_wait_sleep(&pv_done[(q - 1) & 1], ((q - 1) >> 1) & 1, c.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) {
                     alive = false;
                     continue;
                 }
                 tc_fence_after();
-                float ov[64];
-                tmem_ld64(lane_base + kColO + 64 * hf, ov);
+                float ov[kOCols];
+                tmem_ld_n<kOCols>(lane_base + kColO + kOCols * cq, ov);
+                uint32_t ou[kOCols];
 #pragma unroll
-                for (int e = 0; e < 64; ++e) ov[e] *= rescale ? alpha : 1.f;
-                tmem_st64(lane_base + kColO + 64 * hf, ov);
+                for (int e = 0; e < kOCols; ++e) ou[e] = __float_as_uint(ov[e] * (rescale ? alpha : 1.f));
+                tmem_st_n<kOCols>(lane_base + kColO + kOCols * cq, ou);
             }
-            uint8_t* prow = dyn + kOffP + (q & 1) * 32768 + r * 128;
-#pragma unroll
-            for (int cch = 0; cch < 4; ++cch) {
-                const int off = (((4 * hf + cch) ^ (r & 7)) << 4);
-                *reinterpret_cast<uint4*>(prow + off) = make_uint4(ph[4 * cch], ph[4 * cch + 1], ph[4 * cch + 2], ph[4 * cch + 3]);
-                *reinterpret_cast<uint4*>(prow + 16384 + off) =
-                    make_uint4(pl[4 * cch], pl[4 * cch + 1], pl[4 * cch + 2], pl[4 * cch + 3]);
-            }
-            fence_proxy_async_smem();
+            // this group's tokens: kCols / 2 columns of hi pairs, as many of lo pairs
+            const uint32_t tP = lane_base + kColP + 64 * (q & 1) + (kCols / 2) * cq;
+            tmem_st_n<kCols / 2>(tP, ph);
+            tmem_st_n<kCols / 2>(tP + 32, pl);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[q & 1]);
         }
-        // the split's normalised output of this row: this warp's 64 channels
-        xl[hf][r] = l;
-        named_bar(1 + qd, 64);
-        const float lt = xl[0][r] + xl[1][r];
-        float ov[64];
+        // the split's normalised output of this row: this warp's kOCols channels
+        xl[cq][r] = l;
+        named_bar(1 + qd, 32 * kCq);
+        float lt = 0.f;
+#pragma unroll
+        for (int x = 0; x < kCq; ++x) lt += xl[x][r];
+        float ov[kOCols];
         bool have = false;
         if (alive && nproc > 0) {
             bool ok = true;
@@ -546,21 +599,21 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             have = __shfl_sync(0xffffffffu, ok, 0);
             if (have) {
                 tc_fence_after();
-                tmem_ld64(lane_base + kColO + 64 * hf, ov);
+                tmem_ld_n<kOCols>(lane_base + kColO + kOCols * cq, ov);
             }
         }
         if (gr < R) {
             const int ti = gr / G, g = gr % G;
             const int64_t orow = (((int64_t)s * a.M + ti) * c.H_q + h * G + g) * a.num_splits + sp;
-            float* dst = a.o_part + orow * kHeadDim + 64 * hf;
+            float* dst = a.o_part + orow * kHeadDim + kOCols * cq;
             const bool any = have && lt > 0.f;
             const float inv = any ? 1.f / lt : 0.f;
 #pragma unroll
-            for (int e = 0; e < 64; e += 4)
+            for (int e = 0; e < kOCols; e += 4)
                 *reinterpret_cast<float4*>(dst + e) =
                     any ? make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (hf == 0) a.lse_part[orow] = any ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
+            if (cq == 0) a.lse_part[orow] = any ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
         }
     }
     // every role is done with TMEM: the allocating warp releases it

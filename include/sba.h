@@ -37,6 +37,8 @@
  *    (shared-memory limits, cluster sizes).  A cudaDeviceReset discards them
  *    on the device; a process that resets a device reloads the library before
  *    using it there again (calls otherwise fail with SBA_ERR_CUDA).
+ *  - Every softmax_scale argument must be positive and finite
+ *    (SBA_ERR_INVALID_ARG otherwise).
  *  - Data-dependent problems found on the device (a block-table entry outside
  *    [0, num_pages), a position outside the table, a selected index outside
  *    [0, N), a wait that timed out) never trap: the offending access is

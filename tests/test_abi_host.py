@@ -150,6 +150,7 @@ def test_rejects_bad_decode_step_arguments_on_host():
     assert _step(c, out_dtype=7) == E
     assert _step(c, scale=0.0) == E
     assert _step(c, scale=float("nan")) == E
+    assert _step(c, scale=float("inf")) == E
     assert _step(c, n_new=-1) == E
     assert _step(c, n_new=1, k_new=0x1000, v_new=0x2000) == E                 # no positions
     assert _step(c, n_new=1, k_new=None, v_new=0x2000, pos=0x3000) == E
@@ -202,12 +203,14 @@ def test_rejects_bad_multi_token_arguments_on_host():
     assert sdm(ctypes.byref(c), 0x5000, 0, 0x6000, 0x7000, 16, 0.088, 2, 0x8000, 0x9000, None) == E
     assert sdm(ctypes.byref(c), 0x5000, 4, None, 0x7000, 16, 0.088, 2, 0x8000, 0x9000, None) == E
     assert sdm(ctypes.byref(c), 0x5000, 4, 0x6000, 0x7000, 16, 0.0, 2, 0x8000, 0x9000, None) == E
+    assert sdm(ctypes.byref(c), 0x5000, 4, 0x6000, 0x7000, 16, float("inf"), 2, 0x8000, 0x9000, None) == E
     assert sdm(ctypes.byref(c), 0x5000, 4, 0x6000, 0x7000, 16, 0.088, 0, 0x8000, 0x9000, None) == E
     rect = lib.sba_rectify
     assert rect(ctypes.byref(c), 0x5000, 0x1000, 0x2000, 0, 0.088, 2, 0x8000, 0x9000, None) == E
     assert rect(ctypes.byref(c), 0x5000, 0x1000, 0x2000, 129, 0.088, 2, 0x8000, 0x9000, None) == \
-        sba.SBA_ERR_UNSUPPORTED                                                    # window beyond the ring
+        sba.SBA_ERR_UNSUPPORTED                                                    # window beyond f = 128
     assert rect(ctypes.byref(c), 0x5000, None, 0x2000, 32, 0.088, 2, 0x8000, 0x9000, None) == E
+    assert rect(ctypes.byref(c), 0x5000, 0x1000, 0x2000, 32, float("inf"), 2, 0x8000, 0x9000, None) == E
     assert rect(ctypes.byref(c), 0x5000, 0x1008, 0x2000, 32, 0.088, 2, 0x8000, 0x9000, None) == E
     assert lib.sba_multi_row_groups(ctypes.byref(c), 32) == (32 * c.H_q // c.H_kv + 127) // 128
     outer = lib.sba_sparse_decode_outer
