@@ -6,43 +6,44 @@
 // and each of the f tokens attends causally to the whole cache (Key points:
 // f in {16, 32, 64, 128}).  With the M*G query rows of a group sharing every
 // key and value tile, this is a dense contraction: 128 query rows against each
-// 64-token tile, the shape the tensor cores take whole.
+// 128-token tile, the shape the tensor cores take whole.
 //
-// One CTA per (split, KV head x row group of 128 query rows, sequence); 576
-// threads:
-//  - warp 16 (producer) streams each block in 64-token stages (K0 K1 V0 V1: four
-//    2-D TMA loads of 64 rows x 128 B, 128-byte swizzle, no multicast) into a
-//    ring of six 32 KB stages (shared memory holds nothing else: Q and P live in
-//    TMEM).  Before a block the window touches is loaded, it
-//    writes the window's K/V rows of that block into the cache (a proxy fence
-//    orders them ahead of the tile load); after its last fill it recomputes the
-//    Quest min/max of those blocks from their keys.  Rows past len are zeroed in
-//    the stage before anyone reads it.
-//  - warp 17 (MMA) allocates all 512 TMEM columns and, one thread issuing, runs
-//    S = Q K^T for each stage (M 128 rows, N 64 tokens, K 128 channels: eight
-//    tcgen05.mma kind::f16, bf16 in, fp32 accumulate; A = Q from TMEM, B = the
-//    K tile) into one of two TMEM S buffers (columns 0-63, 64-127), so the next
-//    stage's S is computed while the softmax works on this one; then, once P
-//    is written, O += P_hi V + P_lo V (M 128, N 128 channels, K 64 tokens;
-//    A = P from TMEM, V read MN-major straight from the TMA tile) into TMEM
-//    columns 128-255.  tcgen05.commit signals S, O and the stage's release on
+// One CTA per (split, KV head x row group of 128 query rows, sequence): eight
+// softmax warps, a producer warp and an MMA warp.
+//  - the producer warp streams the CTA's share of the sequence in 128-token
+//    stages (K0 K1 V0 V1 halves of 128 rows x 128 B, each filled by two 2-D
+//    TMA loads of 64 rows, 128-byte swizzle, no multicast) into a ring of
+//    three 64 KB stages (shared memory holds nothing else).  Before a block
+//    the window touches is loaded, it writes the window's K/V rows of that
+//    block into the cache (a proxy fence orders them ahead of the tile load);
+//    rows past the share or past len are zeroed in the stage before anyone
+//    reads it; after its last stage it recomputes the Quest min/max of the
+//    touched blocks from their keys in global memory.
+//  - the MMA warp allocates all 512 TMEM columns and, one thread issuing, runs
+//    S = Q K^T for each stage (M 128 rows, N 128 tokens, K 128 channels:
+//    eight tcgen05.mma kind::f16, bf16 in, fp32 accumulate; A = Q from TMEM,
+//    B = the K tile) into one of two S/P buffers (TMEM columns 0-127,
+//    128-255), so the next stage's S is computed while the softmax works on
+//    this one; then, once P has replaced S in the buffer, O += P_hi V + P_lo V
+//    (M 128, N 128 channels, K 128 tokens; A = P from TMEM, V read MN-major
+//    straight from the TMA tile) into TMEM columns 256-383.  The S of stage
+//    q + 2 is issued only after O += P V of stage q has completed (the two
+//    share a buffer).  tcgen05.commit signals S, O and the stage's release on
 //    mbarriers.  A 16-bit A operand in TMEM is row r = lane r with two
 //    consecutive K elements per 32-bit column (the lower one in the low half):
-//    Q takes columns 384-447 (128 channels), each of the two P buffers 64
-//    columns from 256 (32 for the hi parts of its 64 tokens, then 32 for the lo).
-//  - warps 0-15 (softmax): query row r = TMEM lane r is shared by the four
-//    warps w with w % 4 = r / 32, warp w owning columns 16 (w / 4) .. + 15 of
-//    each 64-token stage.  A thread reads its 16 columns of S (tcgen05.ld
-//    32x32b.x16), applies the causal limit (t <= len - f + i for token i),
-//    agrees on the row maximum with the other three warps through shared
-//    memory, keeps an online softmax in base 2 (the scale folded into the
-//    exponent's FMA) whose offset moves only when the row maximum grows by
-//    more than 2^8 (then O's row is rescaled in TMEM; otherwise exponentials
-//    stay below 2^8), and writes its 16 tokens of P as bf16 hi + lo parts
-//    (hi + lo within 2^-15 |p| of p) into one of the two TMEM P buffers
-//    (tcgen05.st).
-//    At the end it reads its 32 columns of O, normalises them and writes the
-//    split's O and LSE ([B][f][H_q][S][d], [B][f][H_q][S]).
+//    Q takes columns 384-447 (128 channels); P the 128 columns of its buffer
+//    (64 for the hi parts of the 128 tokens, then 64 for the lo).
+//  - the softmax warps: query row r = TMEM lane r is shared by the warps w with
+//    w % 4 = r / 32, each owning an equal share of the stage's 128 columns.  A
+//    thread reads its columns of S (tcgen05.ld 32x32b), applies the causal
+//    limit (t <= len - f + i for token i), agrees on the row maximum with the
+//    row's other warps through shared memory, keeps an online softmax in base 2
+//    (the scale folded into the exponent's FMA) whose offset moves only when
+//    the row maximum grows by more than 2^8 (then O's row is rescaled in TMEM;
+//    otherwise exponentials stay below 2^8), and writes its tokens of P as bf16
+//    hi + lo parts (hi + lo within 2^-15 |p| of p) over S in the same buffer
+//    (tcgen05.st).  At the end it reads its columns of O, normalises them and
+//    writes the split's O and LSE ([B][f][H_q][S][d], [B][f][H_q][S]).
 // Every wait is bounded: a wait that runs out reports SBA_DEV_TIMEOUT and the
 // roles stop, and TMEM is released on every path.
 #include <cuda.h>
@@ -64,21 +65,23 @@ bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);  // decod
 namespace {
 
 constexpr int kRtRows = 128;               // query rows per CTA: the MMA's M
-constexpr int kRtStages = 6;               // 64-token K/V stages: 192 KB, all the shared memory there is
-constexpr int kRtStage = 32768;
-constexpr int kRtHalf = 8192;              // 64 rows x 128 B
+constexpr int kStageTok = 128;             // tokens per ring stage: the N of S = Q K^T
+constexpr int kRtStages = 3;               // 64 KB K/V stages: 192 KB, all the shared memory there is
+constexpr int kRtStage = 65536;
+constexpr int kRtHalf = 16384;             // 128 rows x 128 B (64 channels of K or V)
 constexpr int kSmWarps = SBA_RECT_SOFTMAX_WARPS;  // softmax warps: kCq per TMEM lane quarter
 constexpr int kCq = kSmWarps / 4;          // warps sharing a query row (column groups)
-constexpr int kCols = 64 / kCq;            // S columns (tokens) of a stage per thread
+constexpr int kCols = kStageTok / kCq;     // S columns (tokens) of a stage per thread
 constexpr int kOCols = 128 / kCq;          // O (and Q) channels per thread
 constexpr int kRtThreads = (kSmWarps + 2) * 32;  // softmax warps, then the producer, then the MMA warp
 constexpr int kProdWarp = kSmWarps, kMmaWarp = kSmWarps + 1;
 static_assert(kSmWarps == 8 || kSmWarps == 16, "two or four warps per TMEM lane quarter");
+static_assert(kCols % 32 == 0, "P is written 32 tokens at a time");
 constexpr int kRtSmem = kRtStages * kRtStage + 1024;
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S buffers 0-63 and 64-127 (fp32); O 128-255 (fp32); P buffers 256-319 and
-// 320-383 (bf16 pairs: hi parts in the first 32, lo parts in the next 32); Q 384-447 (bf16 pairs)
-constexpr uint32_t kColS = 0, kColO = 128, kColP = 256, kColQ = 384;
+// TMEM columns: S/P buffers 0-127 and 128-255 (S in fp32; then P as bf16 pairs: hi parts in the
+// first 64, lo parts in the next 64); O 256-383 (fp32); Q 384-447 (bf16 pairs)
+constexpr uint32_t kColS = 0, kColO = 256, kColQ = 384;
 
 struct RtArgs {
     sba_cache c;
@@ -219,7 +222,6 @@ template <int kBlk>
 __global__ void __launch_bounds__(kRtThreads, 1)
     rect_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ RtArgs a) {
-    constexpr int kSub = kBlk / 64;
     extern __shared__ uint8_t dyn_raw[];
     uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t kv_full[kRtStages], kv_empty[kRtStages], zbar, q_full, s_full[2], p_full[2], pv_done[2], fin;
@@ -273,14 +275,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     if (!appends && tid == 0 && sp == 0 && blockIdx.y == 0) report(c.status, SBA_DEV_BAD_POSITION);
     const int tb0 = appends ? pos0 / kBlk : N;
     const int i0 = (int)((int64_t)N * sp / a.num_splits), i1 = (int)((int64_t)N * (sp + 1) / a.num_splits);
-    const int nfill = (i1 - i0) * kSub;
-    auto fill_valid = [&](int f) {  // tokens of fill f below len
-        const int j = i0 + f / kSub, sb = f % kSub;
-        return min(64, max(0, len - j * kBlk - 64 * sb));
-    };
-    // only the last block's second half can be empty, and it is the last fill of its share: the
-    // processed fills are fills 0 .. nproc-1 for every role
-    const int nproc = (nfill > 0 && fill_valid(nfill - 1) == 0) ? nfill - 1 : nfill;
+    // the share's tokens [t_begin, t_end) in 128-token stages (every stage holds at least one)
+    const int t_begin = i0 * kBlk, t_end = min(len, i1 * kBlk);
+    const int nproc = t_end > t_begin ? (t_end - t_begin + kStageTok - 1) / kStageTok : 0;
+    auto stage_valid = [&](int q) { return min(kStageTok, t_end - t_begin - kStageTok * q); };
 
     // this thread's share of its query row (row = TMEM lane 32 (warp % 4) + lane, channels
     // kOCols (warp / 4) ..): zero past the group's rows
@@ -313,53 +311,67 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // ------------------------------ producer ------------------------------
         uint32_t zpar = 0;
         for (int q = 0; q < nproc && alive; ++q) {
-            const int vf = fill_valid(q);
-            const int i = i0 + q / kSub, sb = q % kSub, j = i;
+            const int vf = stage_valid(q);  // 1 .. 128 tokens of the stage in the share
             const int st = q % kRtStages;
             if (q >= kRtStages) {
                 if (lane == 0) alive = mbar_wait_sleep(&kv_empty[st], ((q / kRtStages) - 1) & 1, c.status);
                 alive = __shfl_sync(0xffffffffu, alive, 0);
                 if (!alive) break;
             }
-            const int pg = (int)page_of(c, s, j, lane == 0 ? c.status : nullptr);
             uint8_t* base = dyn + (size_t)st * kRtStage;
-            if (pg < 0) {
-                // a bad table entry (reported): the stage is zeros, the roles stay in step
-                for (int e = lane; e < kRtStage / 16; e += 32) reinterpret_cast<uint4*>(base)[e] = make_uint4(0u, 0u, 0u, 0u);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&kv_full[st]);
-                continue;
-            }
-            if (appends && sb == 0 && j >= tb0) {
-                // the window's rows of this block, each lane's stores ordered ahead of the tile load
-                const int t0 = max(pos0, j * kBlk), t1 = min(len, (j + 1) * kBlk);
-                for (int e = lane; e < (t1 - t0) * 32; e += 32) {
-                    const int t = t0 + (e >> 5), half = (e >> 4) & 1, l = e & 15;
-                    const int64_t src = (((int64_t)s * a.M + (t - pos0)) * c.H_kv + h) * 16 + l;
-                    const uint4 v = __ldg((half ? a.v_new : a.k_new) + src);
-                    reinterpret_cast<uint4*>(half ? c.v : c.k)[(((int64_t)pg * c.H_kv + h) * kBlk + t % kBlk) * 16 + l] = v;
+            const int t0 = t_begin + kStageTok * q;
+            // the stage's two 64-row halves: page of each (-1: not loaded), the window's rows of a
+            // block written before its first half is loaded
+            int pgs[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int t = t0 + 64 * h2, j = t / kBlk;
+                pgs[h2] = -1;
+                if (64 * h2 >= vf) continue;
+                pgs[h2] = (int)page_of(c, s, j, lane == 0 ? c.status : nullptr);
+                if (pgs[h2] >= 0 && appends && t % kBlk == 0 && j >= tb0) {
+                    const int w0 = max(pos0, j * kBlk), w1 = min(len, (j + 1) * kBlk);
+                    for (int e = lane; e < (w1 - w0) * 32; e += 32) {
+                        const int tt = w0 + (e >> 5), half = (e >> 4) & 1, l = e & 15;
+                        const int64_t src = (((int64_t)s * a.M + (tt - pos0)) * c.H_kv + h) * 16 + l;
+                        const uint4 v = __ldg((half ? a.v_new : a.k_new) + src);
+                        reinterpret_cast<uint4*>(half ? c.v : c.k)[(((int64_t)pgs[h2] * c.H_kv + h) * kBlk + tt % kBlk) * 16 + l] = v;
+                    }
                 }
-                fence_proxy_async_global();
-                __syncwarp();
             }
-            uint64_t* bar = vf == 64 ? &kv_full[st] : &zbar;
-            if (lane == 0) {
-                const int y = (pg * c.H_kv + h) * kBlk + 64 * sb;
-                mbar_arrive_expect_tx(bar, kRtStage);
-                tma_load_2d(base, &tmK, bar, 0, y);
-                tma_load_2d(base + kRtHalf, &tmK, bar, 64, y);
-                tma_load_2d(base + 2 * kRtHalf, &tmV, bar, 0, y);
-                tma_load_2d(base + 3 * kRtHalf, &tmV, bar, 64, y);
+            fence_proxy_async_global();  // this lane's window rows ahead of the tile loads
+            __syncwarp();
+            const int nload = (pgs[0] >= 0) + (pgs[1] >= 0);
+            // a stage with rows to zero (past the share or len, or a bad table entry, reported) lands on
+            // the side barrier first
+            const bool zero = vf < kStageTok || nload < 2;
+            uint64_t* bar = zero ? &zbar : &kv_full[st];
+            if (lane == 0 && nload > 0) {
+                mbar_arrive_expect_tx(bar, nload * (kRtStage / 2));
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    if (pgs[h2] < 0) continue;
+                    const int t = t0 + 64 * h2;
+                    const int y = (pgs[h2] * c.H_kv + h) * kBlk + t % kBlk;
+                    uint8_t* dst = base + 64 * 128 * h2;
+                    tma_load_2d(dst, &tmK, bar, 0, y);
+                    tma_load_2d(dst + kRtHalf, &tmK, bar, 64, y);
+                    tma_load_2d(dst + 2 * kRtHalf, &tmV, bar, 0, y);
+                    tma_load_2d(dst + 3 * kRtHalf, &tmV, bar, 64, y);
+                }
             }
-            if (vf < 64) {
-                // rows past len may hold anything: zero them before the tensor cores read the stage
+            if (zero) {
+                // rows that are not the share's valid tokens may hold anything (NaN included, or a
+                // previous stage): zero them before the tensor cores read the stage
                 bool ok = true;
-                if (lane == 0) ok = mbar_wait(&zbar, zpar, c.status);
-                zpar ^= 1u;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                for (int e = lane; e < (64 - vf) * 32 && ok; e += 32) {
-                    const int rr = vf + (e >> 5), part = (e >> 4) & 1, ch = e & 15;
+                if (nload > 0) {
+                    if (lane == 0) ok = mbar_wait(&zbar, zpar, c.status);
+                    zpar ^= 1u;
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                }
+                for (int e = lane; e < kStageTok * 32 && ok; e += 32) {
+                    const int rr = e >> 5, part = (e >> 4) & 1, ch = e & 15;  // row, K or V, 16-byte chunk
+                    if (rr < vf && pgs[rr >> 6] >= 0) continue;
                     *reinterpret_cast<uint4*>(base + (2 * part + (ch >> 3)) * kRtHalf + rr * 128 + ((ch & 7) << 4)) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
@@ -406,26 +418,29 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issue ------------------------------
-        constexpr uint32_t kIdQK = umma_idesc(128, 64, false);
+        constexpr uint32_t kIdQK = umma_idesc(128, kStageTok, false);
         constexpr uint32_t kIdPV = umma_idesc(128, 128, true);
         // descriptors of ring stage 0 (K tile: K-major; V tile: MN-major, its two 64-channel halves
-        // 8 KB apart); a stage or a K step adds its byte offset / 16 to the start-address field,
+        // 16 KB apart); a stage or a K step adds its byte offset / 16 to the start-address field,
         // which stays below 2^14 for every shared-memory address
         const uint32_t ring = smem_u32(dyn);
         const uint64_t dK0 = umma_desc(ring, 16, 1024), dV0 = umma_desc(ring + 2 * kRtHalf, kRtHalf, 1024);
         bool issued = false;  // any MMA issued by this warp
         if (lane == 0) alive = mbar_wait_sleep(&q_full, 0, c.status);  // Q in TMEM
         alive = __shfl_sync(0xffffffffu, alive, 0);
-        // S(q) = Q K(q)^T into S buffer q % 2; K = 128 channels in eight steps of 16 (32 bytes
-        // along the swizzled rows)
+        // S(q) = Q K(q)^T into buffer q % 2 once O += P V of stage q - 2 (whose P it holds) has
+        // completed; K = 128 channels in eight steps of 16 (32 bytes along the swizzled rows)
         auto issue_qk = [&](int q) {
             const int st = q % kRtStages;
-            if (lane == 0) alive = mbar_wait_sleep(&kv_full[st], (q / kRtStages) & 1, c.status);
+            if (lane == 0) {
+                alive = mbar_wait_sleep(&kv_full[st], (q / kRtStages) & 1, c.status);
+                if (alive && q >= 2) alive = mbar_wait_sleep(&pv_done[q & 1], ((q - 2) >> 1) & 1, c.status);
+            }
             alive = __shfl_sync(0xffffffffu, alive, 0);
             if (!alive) return;
             tc_fence_after();
             const uint64_t dK = dK0 + (uint64_t)((st * kRtStage) >> 4);
-            const uint32_t tS = tm + kColS + 64 * (q & 1);
+            const uint32_t tS = tm + kColS + 128 * (q & 1);
             if (lane == 0) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -438,8 +453,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         };
         if (nproc > 0 && alive) issue_qk(0);
         for (int q = 0; q < nproc && alive; ++q) {
-            // the next stage's S overlaps this stage's softmax (its S buffer was read by the softmax of
-            // stage q - 1, whose P has been waited for)
+            // the next stage's S overlaps this stage's softmax
             if (q + 1 < nproc) {
                 issue_qk(q + 1);
                 if (!alive) break;
@@ -450,14 +464,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             tc_fence_after();
             const int st = q % kRtStages;
             const uint64_t dV = dV0 + (uint64_t)((st * kRtStage) >> 4);
-            const uint32_t tP = tm + kColP + 64 * (q & 1);
+            const uint32_t tP = tm + kColS + 128 * (q & 1);
             if (lane == 0) {
-                // O += P V: K = 64 tokens in four steps of 16 (two 8-token groups of the V tile, 2 KB)
+                // O += P V: K = 128 tokens in eight steps of 16 (two 8-token groups of the V tile, 2 KB)
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tm + kColO, tP + 32 * part + 8 * kk, dV + (uint64_t)((kk * 2048) >> 4), kIdPV,
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16_ts(tm + kColO, tP + 64 * part + 8 * kk, dV + (uint64_t)((kk * 2048) >> 4), kIdPV,
                                     (q > 0 || part > 0 || kk > 0));
                 umma_commit(&pv_done[q & 1]);
                 umma_commit(&kv_empty[st]);
@@ -484,9 +498,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // (a wait that runs out turns this warp dead; a dead warp still takes every named barrier of the
         // loop, so the row's other warps never wait on it forever, and arrives on nothing)
         for (int q = 0; q < nproc; ++q) {
-            const int vf = fill_valid(q);
-            const int j = i0 + q / kSub, sb = q % kSub;
-            const int base = j * kBlk + 64 * sb + kCols * cq;  // position of this group's first token
+            const int vf = stage_valid(q);
+            const int base = t_begin + kStageTok * q + kCols * cq;  // position of this group's first token
             bool ok = alive;
             if (ok) {
                 if (lane == 0) ok = mbar_wait_sleep(&s_full[q & 1], (q >> 1) & 1, c.status);
@@ -496,7 +509,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             float mx = -INFINITY;
             if (ok) {
                 tc_fence_after();
-                tmem_ld_n<kCols>(lane_base + kColS + 64 * (q & 1) + kCols * cq, sv);
+                tmem_ld_n<kCols>(lane_base + kColS + 128 * (q & 1) + kCols * cq, sv);
                 const int nval = min(kCols, min(vf - kCols * cq, lim - base));  // valid columns of this group
                 if (nval < kCols) {
 #pragma unroll
@@ -530,37 +543,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             const bool rescale = q > 0 && alpha != 1.f;
             // (a row still without a valid token has every score at -inf: offset 0 gives 0 for each)
             const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-            // P = hi + lo in bf16 by integer operations (no conversion instructions): hi = p with its
-            // low 16 bits cleared (truncation), r = p - hi (exact in fp32, 0 <= r < 2^-7 p) rounded to
-            // bf16 for lo by adding half a bf16 unit before its low 16 bits are dropped; the pair's
-            // upper halves are packed by one byte permute.  |p - hi - lo| <= 2^-8 r < 2^-15 p while r
-            // is a normal float (p >= 2^-100); below that the error is under 2^-130, nothing next to
-            // a row sum >= 1.
-            uint32_t ph[kCols / 2], pl[kCols / 2];
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int t = 0; t < kCols; t += 2) {
-                const float p0 = ex2(fmaf(sv[t], sl2, neg_m));
-                const float p1 = ex2(fmaf(sv[t + 1], sl2, neg_m));
-                ls[(t >> 1) & 3] += p0 + p1;
-                const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-                const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
-                const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
-                ph[t / 2] = __byte_perm(u0, u1, 0x7632);
-                pl[t / 2] = __byte_perm(__float_as_uint(r0) + 0x8000u, __float_as_uint(r1) + 0x8000u, 0x7632);
-            }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            // this P buffer is free once O += P V of stage q - 2 has completed; O itself (to rescale)
-            // once that of stage q - 1 has
-            if (q >= 2) {
-                if (lane == 0) ok = mbar_wait_sleep(&pv_done[q & 1], ((q - 2) >> 1) & 1, c.status);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) {
-                    alive = false;
-                    continue;
-                }
-                tc_fence_after();
-            }
+            // O (to rescale) once O += P V of stage q - 1 has completed
             if (__any_sync(0xffffffffu, rescale)) {
                 if (lane == 0) ok = mbar_wait_sleep(&pv_done[(q - 1) & 1], ((q - 1) >> 1) & 1, c.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -569,17 +552,45 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                     continue;
                 }
                 tc_fence_after();
-                float ov[kOCols];
-                tmem_ld_n<kOCols>(lane_base + kColO + kOCols * cq, ov);
-                uint32_t ou[kOCols];
+                const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < kOCols; c0 += 16) {  // 16 columns at a time (few registers)
+                    float ov[16];
+                    tmem_ld16(lane_base + kColO + kOCols * cq + c0, ov);
+                    uint32_t ou[16];
 #pragma unroll
-                for (int e = 0; e < kOCols; ++e) ou[e] = __float_as_uint(ov[e] * (rescale ? alpha : 1.f));
-                tmem_st_n<kOCols>(lane_base + kColO + kOCols * cq, ou);
+                    for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(ov[e] * f);
+                    tmem_st16(lane_base + kColO + kOCols * cq + c0, ou);
+                }
             }
-            // this group's tokens: kCols / 2 columns of hi pairs, as many of lo pairs
-            const uint32_t tP = lane_base + kColP + 64 * (q & 1) + (kCols / 2) * cq;
-            tmem_st_n<kCols / 2>(tP, ph);
-            tmem_st_n<kCols / 2>(tP + 32, pl);
+            // P = hi + lo in bf16 by integer operations (no conversion instructions): hi = p with its
+            // low 16 bits cleared (truncation), r = p - hi (exact in fp32, 0 <= r < 2^-7 p) rounded to
+            // bf16 for lo by adding half a bf16 unit before its low 16 bits are dropped; the pair's
+            // upper halves are packed by one byte permute.  |p - hi - lo| <= 2^-8 r < 2^-15 p while r
+            // is a normal float (p >= 2^-100); below that the error is under 2^-130, nothing next to
+            // a row sum >= 1.  Every warp of the row has read its S before the barrier above, so P may
+            // replace S anywhere in the buffer: this group's tokens go to kCols / 2 columns of hi pairs
+            // from (kCols / 2) cq and as many of lo pairs 64 columns further, 32 tokens at a time.
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t tP = lane_base + kColS + 128 * (q & 1) + (kCols / 2) * cq;
+#pragma unroll
+            for (int c0 = 0; c0 < kCols; c0 += 32) {
+                uint32_t ph[16], pl[16];
+#pragma unroll
+                for (int t = 0; t < 32; t += 2) {
+                    const float p0 = ex2(fmaf(sv[c0 + t], sl2, neg_m));
+                    const float p1 = ex2(fmaf(sv[c0 + t + 1], sl2, neg_m));
+                    ls[(t >> 1) & 3] += p0 + p1;
+                    const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                    const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
+                    const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                    ph[t / 2] = __byte_perm(u0, u1, 0x7632);
+                    pl[t / 2] = __byte_perm(__float_as_uint(r0) + 0x8000u, __float_as_uint(r1) + 0x8000u, 0x7632);
+                }
+                tmem_st16(tP + c0 / 2, ph);
+                tmem_st16(tP + 64 + c0 / 2, pl);
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -591,30 +602,31 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         float lt = 0.f;
 #pragma unroll
         for (int x = 0; x < kCq; ++x) lt += xl[x][r];
-        float ov[kOCols];
         bool have = false;
         if (alive && nproc > 0) {
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&pv_done[(nproc - 1) & 1], ((nproc - 1) >> 1) & 1, c.status);
             have = __shfl_sync(0xffffffffu, ok, 0);
-            if (have) {
-                tc_fence_after();
-                tmem_ld_n<kOCols>(lane_base + kColO + kOCols * cq, ov);
+            if (have) tc_fence_after();
+        }
+        const int ti = gr / G, g = gr % G;
+        const int64_t orow = (((int64_t)s * a.M + ti) * c.H_q + h * G + g) * a.num_splits + sp;
+        const bool any = have && lt > 0.f;
+        const float inv = any ? 1.f / lt : 0.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kOCols; c0 += 32) {  // (the loads are warp-collective: every lane takes them)
+            float ov[32];
+            if (have) tmem_ld32(lane_base + kColO + kOCols * cq + c0, ov);
+            if (gr < R) {
+                float* dst = a.o_part + orow * kHeadDim + kOCols * cq + c0;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(dst + e) =
+                        any ? make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-        if (gr < R) {
-            const int ti = gr / G, g = gr % G;
-            const int64_t orow = (((int64_t)s * a.M + ti) * c.H_q + h * G + g) * a.num_splits + sp;
-            float* dst = a.o_part + orow * kHeadDim + kOCols * cq;
-            const bool any = have && lt > 0.f;
-            const float inv = any ? 1.f / lt : 0.f;
-#pragma unroll
-            for (int e = 0; e < kOCols; e += 4)
-                *reinterpret_cast<float4*>(dst + e) =
-                    any ? make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv, ov[e + 3] * inv)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (cq == 0) a.lse_part[orow] = any ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
-        }
+        if (gr < R && cq == 0) a.lse_part[orow] = any ? (m_used + log2f(lt)) * kLn2 : -INFINITY;
     }
     // every role is done with TMEM: the allocating warp releases it
     tc_fence_before();
