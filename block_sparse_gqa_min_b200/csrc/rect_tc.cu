@@ -27,9 +27,9 @@
 //    this one; then, once P has replaced S in the buffer, O += P_hi V + P_lo V
 //    (M 128, N 128 channels, K 128 tokens; A = P from TMEM, V read MN-major
 //    straight from the TMA tile) into TMEM columns 256-383.  The S of stage
-//    q + 2 is issued only after O += P V of stage q has completed (the two
-//    share a buffer).  tcgen05.commit signals S, O and the stage's release on
-//    mbarriers.  A 16-bit A operand in TMEM is row r = lane r with two
+//    q + 2 overwrites the P that O += P V of stage q reads; the tensor core
+//    runs one thread's MMAs in issue order, so no wait separates them.
+//    tcgen05.commit signals S, O and the stage's release on mbarriers.  A 16-bit A operand in TMEM is row r = lane r with two
 //    consecutive K elements per 32-bit column (the lower one in the low half):
 //    Q takes columns 384-447 (128 channels); P the 128 columns of its buffer
 //    (64 for the hi parts of the 128 tokens, then 64 for the lo).
@@ -428,14 +428,13 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         bool issued = false;  // any MMA issued by this warp
         if (lane == 0) alive = mbar_wait_sleep(&q_full, 0, c.status);  // Q in TMEM
         alive = __shfl_sync(0xffffffffu, alive, 0);
-        // S(q) = Q K(q)^T into buffer q % 2 once O += P V of stage q - 2 (whose P it holds) has
-        // completed; K = 128 channels in eight steps of 16 (32 bytes along the swizzled rows)
+        // S(q) = Q K(q)^T into buffer q % 2; K = 128 channels in eight steps of 16 (32 bytes along
+        // the swizzled rows).  The buffer still holds P of stage q - 2, read by O += P V of that
+        // stage, which this thread issued earlier: the tensor core runs one thread's MMAs in issue
+        // order, so that read comes first without a wait.
         auto issue_qk = [&](int q) {
             const int st = q % kRtStages;
-            if (lane == 0) {
-                alive = mbar_wait_sleep(&kv_full[st], (q / kRtStages) & 1, c.status);
-                if (alive && q >= 2) alive = mbar_wait_sleep(&pv_done[q & 1], ((q - 2) >> 1) & 1, c.status);
-            }
+            if (lane == 0) alive = mbar_wait_sleep(&kv_full[st], (q / kRtStages) & 1, c.status);
             alive = __shfl_sync(0xffffffffu, alive, 0);
             if (!alive) return;
             tc_fence_after();
