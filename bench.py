@@ -135,9 +135,10 @@ def bf16_peak():
         return 1590.0, "fallback"
 
 
-# sources of the fused step kernel: a recorded ncu traffic figure is valid only while they are unchanged
+# sources of each profiled kernel: a recorded ncu traffic figure is valid only while they are unchanged
 KERNEL_SOURCES = {
     "decode_step": ["fused_step.cu", "decode_tile.cuh", "select.cuh", "common.cuh", "launch.cuh"],
+    "rectify": ["rect_tc.cu", "common.cuh", "launch.cuh"],
 }
 
 
@@ -461,6 +462,9 @@ def native(args, rank, world, local, w=None, sweep=False):
                            "frac_executed": round(fe / (r_ms * 1e-3) / 1e12 / tc, 4)},
                 "num_splits": S_r, "row_groups": rg,
                 "kernels": "rect_tc_kernel (tcgen05) + combine_kernel per layer (one CUDA graph)"}
+        rt = recorded_traffic("rectify", w.name)
+        rect["traffic_per_layer"] = rt
+        rect["traffic_over_algorithmic"] = round(rt / (rb / n_layers), 3) if rt else None
         del rgraph
 
     def step():
