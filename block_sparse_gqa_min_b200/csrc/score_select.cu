@@ -116,31 +116,55 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
 
     const int qt = lane & 3, sub = lane >> 2;
     if (kScorer == SBA_SCORER_QUEST) {
-        // coefficients of this lane's 64 descriptor values: qt 0/1 = min row
-        // channels 0-63/64-127 (weights M), qt 2/3 = max row (weights P).
-        const int ch0 = (qt & 1) * 64;
-        const bool use_max = qt >= 2;
-        float coef[64];
+        // the group's coefficients P_c = sum of max(q_c, 0) and M_c = sum of min(q_c, 0) over its
+        // query rows (several query tokens of a sequence: their heads join the group's sum, ReSA
+        // Summary), by the whole CTA: thread t takes channels 8 (t / 16) .. + 7 of every 16th row
+        // from row t % 16 (16-byte loads), the 16 row lanes of a half warp summed by shuffles
+        static_assert(kThreads == 256, "16 channel groups x 16 row lanes");
+        __shared__ float coef_pm[2][kHeadDim];  // [P, M][channel]
+        {
+            const int cg = tid >> 4, rl = tid & 15;
+            float pp[8], mm[8];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) coef[e] = 0.f;
-        // (several query tokens of a sequence: their heads join the group's sum, ReSA Summary)
-        for (int gi = 0; gi < G * a.M; ++gi) {
-            const int g = gi % G, qi = gi / G;
-            const uint4* qp = reinterpret_cast<const uint4*>(
-                a.q + (((int64_t)s * a.M + qi) * c.H_q + h * G + g) * kHeadDim + ch0);
-#pragma unroll
-            for (int k8 = 0; k8 < 8; ++k8) {
-                const uint4 w = __ldg(qp + k8);
+            for (int e = 0; e < 8; ++e) pp[e] = mm[e] = 0.f;
+            const int R = G * a.M;
+#pragma unroll 4
+            for (int gi = rl; gi < R; gi += 16) {
+                const int g = gi % G, qi = gi / G;
+                const uint4 w = __ldg(reinterpret_cast<const uint4*>(
+                    a.q + (((int64_t)s * a.M + qi) * c.H_q + h * G + g) * kHeadDim) + cg);
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float x0 = bf16_lo(ws[e]), x1 = bf16_hi(ws[e]);
-                    coef[8 * k8 + 2 * e] += use_max ? fmaxf(x0, 0.f) : fminf(x0, 0.f);
-                    coef[8 * k8 + 2 * e + 1] += use_max ? fmaxf(x1, 0.f) : fminf(x1, 0.f);
+                    pp[2 * e] += fmaxf(x0, 0.f);
+                    mm[2 * e] += fminf(x0, 0.f);
+                    pp[2 * e + 1] += fmaxf(x1, 0.f);
+                    mm[2 * e + 1] += fminf(x1, 0.f);
                 }
             }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pp[e] += __shfl_xor_sync(0xffffffffu, pp[e], o);
+                    mm[e] += __shfl_xor_sync(0xffffffffu, mm[e], o);
+                }
+            if (rl == 0)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    coef_pm[0][8 * cg + e] = pp[e];
+                    coef_pm[1][8 * cg + e] = mm[e];
+                }
         }
-        __syncthreads();  // pages_s ready
+        __syncthreads();  // coefficients (and pages_s) ready
+        // this lane's 64 descriptor values: qt 0/1 = min row channels 0-63/64-127 (weights M),
+        // qt 2/3 = max row (weights P)
+        const int ch0 = (qt & 1) * 64;
+        const float* cf = coef_pm[qt >= 2 ? 0 : 1] + ch0;
+        float coef[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) coef[e] = cf[e];
         const uint4* desc = reinterpret_cast<const uint4*>(c.desc);
         float* out = a.scores + ((int64_t)s * c.H_kv + h) * mb;
         for (int base = j0 + warp * kBlocksPerWarpIter; base < j1; base += kWarps * kBlocksPerWarpIter) {
