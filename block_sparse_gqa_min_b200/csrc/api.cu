@@ -101,6 +101,11 @@ const char* sba_last_cuda_error(void) {
     return e == cudaSuccess ? "no error" : cudaGetErrorString(e);
 }
 
+int sba_selftest_wait_timeout(int32_t* status, uint64_t limit_ns, void* stream) {
+    if (!status || limit_ns == 0 || limit_ns > 10000000000ull) return SBA_ERR_INVALID_ARG;
+    return after_launch(launch_wait_timeout_selftest(status, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t sba_num_selected(int32_t N, const sba_select_params* p) {
     if (!p) return -1;
     return num_selected(N, *p);

@@ -93,6 +93,7 @@ int launch_multi_query(const sba_cache& c, const void* q, int M, const int32_t* 
 int launch_rectify_tc(const sba_cache& c, const void* q, int f, const void* k_new, const void* v_new, float scale,
                       int num_splits, float* o_part, float* lse_part, cudaStream_t stream);
 int launch_fold_gate(const float* Wq, const float* Wk, int dg, float* A, cudaStream_t stream);
+int launch_wait_timeout_selftest(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
 int launch_combine(const float* o_part, const float* lse_part, int B, int H_q, int S, void* out, int out_dtype,
                    float* lse_out, cudaStream_t stream);
 

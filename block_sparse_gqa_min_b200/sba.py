@@ -112,6 +112,7 @@ _SIGS = {
     "sba_combine": ([_P, _P, _I, _I, _I, _I, _P, _I, _P, _P], ctypes.c_int),
     "sba_fold_gate": ([ctypes.POINTER(sba_gate), _P, _P], ctypes.c_int),
     "sba_static_scratch_bytes": ([], ctypes.c_size_t),
+    "sba_selftest_wait_timeout": ([_P, ctypes.c_uint64, _P], ctypes.c_int),
     "sba_score_select_static": ([ctypes.POINTER(sba_cache), _P, ctypes.POINTER(sba_select_params), _P, _P, _P, _I,
                                  _P], ctypes.c_int),
     "sba_decode_step_cluster": ([ctypes.POINTER(sba_cache), ctypes.POINTER(sba_select_params)], _I),
@@ -343,6 +344,13 @@ def sba_combine(o_part: torch.Tensor, lse_part: torch.Tensor, out: torch.Tensor,
 def sba_fold_gate(Wq: torch.Tensor, Wk: torch.Tensor, A: torch.Tensor, stream=None):
     _check(load().sba_fold_gate(ctypes.byref(sba_gate(_ptr(Wq), _ptr(Wk), int(Wq.shape[0]))), _ptr(A),
                                 _stream(stream)), "sba_fold_gate")
+
+
+def sba_selftest_wait_timeout(status: torch.Tensor, limit_ns: int, stream=None):
+    """Let one bounded wait run out on purpose (nothing arrives on its barrier): SBA_DEV_TIMEOUT
+    is OR-ed into the int32 device `status`, the kernel returns."""
+    _check(load().sba_selftest_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)),
+           "sba_selftest_wait_timeout")
 
 
 def sba_decode_step_cluster(c: Cache, p: sba_select_params) -> int:

@@ -169,6 +169,14 @@ const char *sba_status_string(int status);
  * ("no error" if none); static string, never NULL. */
 const char *sba_last_cuda_error(void);
 
+/* Self-test of the bounded waits every kernel uses (failure detection without
+ * a fault): one warp waits, with the library's own bounded mbarrier wait limited
+ * to limit_ns, on a barrier that nothing arrives on; the wait runs out, ORs
+ * SBA_DEV_TIMEOUT into *status (device int32) and the kernel returns, leaving
+ * the context usable.  0 < limit_ns <= 10 s (SBA_ERR_INVALID_ARG otherwise, or
+ * for a NULL status).  The kernels' own waits give up after about 2 s. */
+int sba_selftest_wait_timeout(int32_t *status, uint64_t limit_ns, void *stream);
+
 /* Host helper: blocks selected for a sequence of N blocks under `p` (the rule
  * above).  Returns -1 if p is NULL. */
 int32_t sba_num_selected(int32_t N, const sba_select_params *p);

@@ -215,3 +215,11 @@ def test_rejects_bad_multi_token_arguments_on_host():
     assert lib.sba_multi_row_groups(ctypes.byref(c), 32) == (32 * c.H_q // c.H_kv + 127) // 128
     outer = lib.sba_sparse_decode_outer
     assert outer(ctypes.byref(c), 0x5000, 0x6000, 0x7000, None, 16, 0.088, 2, 0x8000, 0x9000, None) == E  # needs g
+
+
+def test_rejects_bad_selftest_arguments_on_host():
+    lib = sba.load()
+    E = sba.SBA_ERR_INVALID_ARG
+    assert lib.sba_selftest_wait_timeout(None, 1000, None) == E
+    assert lib.sba_selftest_wait_timeout(0x1000, 0, None) == E
+    assert lib.sba_selftest_wait_timeout(0x1000, 10_000_000_001, None) == E
