@@ -127,6 +127,8 @@ FUSED_GATE_CASES = [
     dict(H_q=5, H_kv=1, b=64, len_lo=65, len_hi=65, n_budget=4, n_local=2),          # C = 1 historical
     dict(H_q=8, H_kv=4, b=128, len_lo=200, len_hi=5000, B=3, n_budget=5, n_local=0, paged=True),
     dict(H_q=10, H_kv=2, b=64, len_lo=300, len_hi=6000, B=3, n_budget=6, n_local=2),  # contiguous, lengths differ
+    dict(H_q=32, H_kv=2, b=128, len_lo=9000, len_hi=9000, n_budget=8, n_local=2),      # G 16: two 8-head tiles
+    dict(H_q=32, H_kv=2, b=64, len_lo=2000, len_hi=9000, B=2, n_budget=10, n_local=1, paged=True),  # G 16, paged
 ]
 
 
@@ -167,10 +169,11 @@ GATE_VARIANTS = [(pos, act) for pos in ("inner", "outer") for act in ("softmax",
 
 
 @pytest.mark.parametrize("pos,act", GATE_VARIANTS)
-@pytest.mark.parametrize("case", [0, 1])
+@pytest.mark.parametrize("case", [0, 1, 2])
 def test_fused_gate_variants(pos, act, case):
     shapes = [dict(H_q=40, H_kv=8, b=64, len_lo=30000, len_hi=30000, n_budget=32, n_local=2, n_min=16),
-              dict(H_q=10, H_kv=2, b=64, len_lo=3000, len_hi=7000, B=2, n_budget=6, n_local=2, paged=True)]
+              dict(H_q=10, H_kv=2, b=64, len_lo=3000, len_hi=7000, B=2, n_budget=6, n_local=2, paged=True),
+              dict(H_q=32, H_kv=2, b=128, len_lo=5000, len_hi=9000, B=2, n_budget=8, n_local=1)]
     w = small_workload(d=128, scorer="gate", dg=128, gate_position=pos, gate_act=act, **shapes[case])
     run_fused(w, seed=11 + case, n_app=1)
 

@@ -110,6 +110,16 @@ def test_multi_query_rows_beyond_one_cta():
     run_multi(w, 20, seed=3)
 
 
+@pytest.mark.parametrize("M,shape", [
+    (128, dict(H_q=8, H_kv=2, b=64, len_lo=3000, len_hi=3000, n_budget=16, n_local=2)),     # 512 rows, 4 row groups
+    (1024, dict(H_q=2, H_kv=2, b=128, len_lo=2100, len_hi=4000, B=2, n_budget=8, n_local=2,
+                paged=True)),                                                                # M at its limit, G 1
+])
+def test_multi_query_many_rows(M, shape):
+    w = small_workload(d=128, **shape)
+    run_multi(w, M, seed=M)
+
+
 def test_multi_query_short_sequences():
     """Sequences shorter than a block and exactly M tokens long (every token a query)."""
     w = small_workload(d=128, H_q=8, H_kv=2, b=64, len_lo=4, len_hi=70, B=4, n_budget=2, n_local=1, paged=True)
@@ -166,6 +176,8 @@ RECT_CASES = [
     (dict(H_q=4, H_kv=1, b=64, len_lo=64, len_hi=64, n_local=1), 64),               # every token new
     (dict(H_q=8, H_kv=2, b=128, len_lo=1000, len_hi=1000, n_local=2), 128),         # 128 tokens over 2 blocks
     (dict(H_q=32, H_kv=2, b=64, len_lo=3000, len_hi=3000, n_local=2), 16),          # 256 rows: 2 row groups
+    (dict(H_q=16, H_kv=1, b=128, len_lo=4000, len_hi=9000, B=2, n_local=2, paged=True), 32),  # G 16: 4 row groups
+    (dict(H_q=7, H_kv=1, b=64, len_lo=129, len_hi=129, n_local=1), 128),            # f = 128 over 3 blocks, 896 rows
 ]
 
 
