@@ -90,6 +90,9 @@ int mq_row_groups(const sba_cache& c, int M);
 int launch_multi_query(const sba_cache& c, const void* q, int M, const int32_t* sel_idx, const int32_t* sel_cnt,
                        int n_max, float scale, int num_splits,
                        float* o_part, float* lse_part, cudaStream_t stream);
+int launch_multi_query_tc(const sba_cache& c, const void* q, int M, const int32_t* sel_idx, const int32_t* sel_cnt,
+                          int n_max, float scale, int num_splits, float* o_part, float* lse_part,
+                          cudaStream_t stream);
 int launch_rectify_tc(const sba_cache& c, const void* q, int f, const void* k_new, const void* v_new, float scale,
                       int num_splits, float* o_part, float* lse_part, cudaStream_t stream);
 int launch_fold_gate(const float* Wq, const float* Wk, int dg, float* A, cudaStream_t stream);

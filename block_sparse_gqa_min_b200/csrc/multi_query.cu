@@ -40,6 +40,7 @@ bool make_kv_tmap(CUtensorMap* m, void* base, uint64_t rows, int blk);  // decod
 namespace {
 
 constexpr int kRowsPerCta = 128;           // 8 row tiles of 16
+constexpr int kTcRows = 64;                // query rows per group from which the tcgen05 kernel serves the call
 constexpr int kMaxConsumers = 8;
 constexpr int kMqThreads = (kMaxConsumers + 1) * 32;
 constexpr int kMqStages = 6;
@@ -400,6 +401,9 @@ int mq_row_groups(const sba_cache& c, int M) {
 int launch_multi_query(const sba_cache& c, const void* q, int M, const int32_t* sel_idx, const int32_t* sel_cnt,
                        int n_max, float scale, int num_splits,
                        float* o_part, float* lse_part, cudaStream_t stream) {
+    // from 64 query rows per group on, the tcgen05 pipeline (rect_tc.cu) takes the same call
+    if (M * (c.H_q / c.H_kv) >= kTcRows)
+        return launch_multi_query_tc(c, q, M, sel_idx, sel_cnt, n_max, scale, num_splits, o_part, lse_part, stream);
     MqArgs a{};
     a.c = c;
     a.q = reinterpret_cast<const __nv_bfloat16*>(q);

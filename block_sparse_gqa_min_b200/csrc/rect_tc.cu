@@ -8,6 +8,12 @@
 // key and value tile, this is a dense contraction: 128 query rows against each
 // 128-token tile, the shape the tensor cores take whole.
 //
+// The same pipeline serves several query tokens sharing one selection
+// (sba_sparse_decode_multi at M*G >= 64 query rows, ReSA Key points: the
+// self-speculative comparison checks several draft tokens with one sparse
+// pass): the block list is then the group's selection, two 64-token blocks or
+// one 128-token block per stage, and nothing is written to the cache.
+//
 // One CTA per (split, KV head x row group of 128 query rows, sequence): eight
 // softmax warps, a producer warp and an MMA warp.
 //  - the producer warp streams the CTA's share of the sequence in 128-token
@@ -86,9 +92,12 @@ constexpr uint32_t kColS = 0, kColO = 256, kColQ = 384;
 struct RtArgs {
     sba_cache c;
     const __nv_bfloat16* q;  // [B][f][H_q][d]
-    int M;                   // f
-    const uint4* k_new;      // [B][f][H_kv][d]: keys and values of positions len-f .. len-1
+    int M;                   // f (the query tokens)
+    const uint4* k_new;      // dense: [B][f][H_kv][d], keys and values of positions len-f .. len-1
     const uint4* v_new;
+    const int32_t* sel_idx;  // sparse: [B][H_kv][n_max], the group's selected blocks
+    const int32_t* sel_cnt;  // sparse: [B][H_kv]
+    int n_max;
     float scale_log2;
     int num_splits;
     float* o_part;           // [B][f][H_q][S][d]
@@ -218,7 +227,7 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
     return d;
 }
 
-template <int kBlk>
+template <int kBlk, bool kSparse>
 __global__ void __launch_bounds__(kRtThreads, 1)
     rect_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ RtArgs a) {
@@ -270,15 +279,42 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         N = c.max_blocks;
         len = N * kBlk;
     }
-    const int pos0 = len - a.M;  // first window token's position
-    const bool appends = a.M > 0 && pos0 >= 0;
-    if (!appends && tid == 0 && sp == 0 && blockIdx.y == 0) report(c.status, SBA_DEV_BAD_POSITION);
+    const int pos0 = len - a.M;  // first query token's position
+    const bool appends = !kSparse && a.M > 0 && pos0 >= 0;
+    if (!kSparse && !appends && tid == 0 && sp == 0 && blockIdx.y == 0) report(c.status, SBA_DEV_BAD_POSITION);
     const int tb0 = appends ? pos0 / kBlk : N;
-    const int i0 = (int)((int64_t)N * sp / a.num_splits), i1 = (int)((int64_t)N * (sp + 1) / a.num_splits);
-    // the share's tokens [t_begin, t_end) in 128-token stages (every stage holds at least one)
+    // dense: the blocks [0, N); sparse: the group's selection, in C-order of the list
+    const int32_t* sel = kSparse ? a.sel_idx + ((int64_t)s * c.H_kv + h) * a.n_max : nullptr;
+    int cnt = N;
+    if (kSparse) {
+        cnt = __ldg(a.sel_cnt + s * c.H_kv + h);
+        if (cnt < 0 || cnt > a.n_max) {
+            if (tid == 0 && sp == 0 && rg == 0) report(c.status, SBA_DEV_BAD_SELECTION);
+            cnt = cnt < 0 ? 0 : a.n_max;
+        }
+    }
+    const int i0 = (int)((int64_t)cnt * sp / a.num_splits), i1 = (int)((int64_t)cnt * (sp + 1) / a.num_splits);
+    // dense: the share's tokens [t_begin, t_end) in 128-token stages (every stage holds at least
+    // one); sparse: the share's blocks, two (b = 64) or one (b = 128) per stage
     const int t_begin = i0 * kBlk, t_end = min(len, i1 * kBlk);
-    const int nproc = t_end > t_begin ? (t_end - t_begin + kStageTok - 1) / kStageTok : 0;
-    auto stage_valid = [&](int q) { return min(kStageTok, t_end - t_begin - kStageTok * q); };
+    const int nproc = kSparse ? (kBlk == 64 ? (i1 - i0 + 1) / 2 : i1 - i0)
+                              : (t_end > t_begin ? (t_end - t_begin + kStageTok - 1) / kStageTok : 0);
+    // 64-token half h2 of stage q: its block j, the position of its first token, and its valid
+    // tokens (0: no such half, or a selected index outside [0, N))
+    auto stage_half = [&](int q, int h2, int& j, int& base) -> int {
+        if (kSparse) {
+            const int idx = kBlk == 64 ? i0 + 2 * q + h2 : i0 + q;
+            if (idx >= i1) return 0;
+            j = __ldg(sel + idx);
+            if (j < 0 || j >= N) return 0;
+            base = j * kBlk + (kBlk == 64 ? 0 : 64 * h2);
+            return max(0, min(64, len - base));
+        } else {
+            base = t_begin + kStageTok * q + 64 * h2;
+            j = base / kBlk;
+            return max(0, min(64, t_end - base));
+        }
+    };
 
     // this thread's share of its query row (row = TMEM lane 32 (warp % 4) + lane, channels
     // kOCols (warp / 4) ..): zero past the group's rows
@@ -311,7 +347,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // ------------------------------ producer ------------------------------
         uint32_t zpar = 0;
         for (int q = 0; q < nproc && alive; ++q) {
-            const int vf = stage_valid(q);  // 1 .. 128 tokens of the stage in the share
             const int st = q % kRtStages;
             if (q >= kRtStages) {
                 if (lane == 0) alive = mbar_wait_sleep(&kv_empty[st], ((q / kRtStages) - 1) & 1, c.status);
@@ -319,16 +354,22 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 if (!alive) break;
             }
             uint8_t* base = dyn + (size_t)st * kRtStage;
-            const int t0 = t_begin + kStageTok * q;
-            // the stage's two 64-row halves: page of each (-1: not loaded), the window's rows of a
-            // block written before its first half is loaded
-            int pgs[2];
+            // the stage's two 64-row halves: valid tokens and page of each (-1: not loaded), the
+            // window's rows of a block written before its first half is loaded (dense)
+            int pgs[2], vh[2], ys[2];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-                const int t = t0 + 64 * h2, j = t / kBlk;
+                int j = 0, t = 0;
+                vh[h2] = stage_half(q, h2, j, t);
                 pgs[h2] = -1;
-                if (64 * h2 >= vf) continue;
+                ys[h2] = 0;
+                if (kSparse && lane == 0 && vh[h2] == 0) {
+                    const int idx = kBlk == 64 ? i0 + 2 * q + h2 : i0 + q;
+                    if (idx < i1 && (j < 0 || j >= N)) report(c.status, SBA_DEV_BAD_SELECTION);
+                }
+                if (vh[h2] == 0) continue;
                 pgs[h2] = (int)page_of(c, s, j, lane == 0 ? c.status : nullptr);
+                ys[h2] = (max(pgs[h2], 0) * c.H_kv + h) * kBlk + t % kBlk;
                 if (pgs[h2] >= 0 && appends && t % kBlk == 0 && j >= tb0) {
                     const int w0 = max(pos0, j * kBlk), w1 = min(len, (j + 1) * kBlk);
                     for (int e = lane; e < (w1 - w0) * 32; e += 32) {
@@ -342,17 +383,16 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             fence_proxy_async_global();  // this lane's window rows ahead of the tile loads
             __syncwarp();
             const int nload = (pgs[0] >= 0) + (pgs[1] >= 0);
-            // a stage with rows to zero (past the share or len, or a bad table entry, reported) lands on
-            // the side barrier first
-            const bool zero = vf < kStageTok || nload < 2;
+            // a stage with rows to zero (past the share or len, a missing half, or a bad table entry,
+            // reported) lands on the side barrier first
+            const bool zero = vh[0] < 64 || vh[1] < 64 || nload < 2;
             uint64_t* bar = zero ? &zbar : &kv_full[st];
             if (lane == 0 && nload > 0) {
                 mbar_arrive_expect_tx(bar, nload * (kRtStage / 2));
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     if (pgs[h2] < 0) continue;
-                    const int t = t0 + 64 * h2;
-                    const int y = (pgs[h2] * c.H_kv + h) * kBlk + t % kBlk;
+                    const int y = ys[h2];
                     uint8_t* dst = base + 64 * 128 * h2;
                     tma_load_2d(dst, &tmK, bar, 0, y);
                     tma_load_2d(dst + kRtHalf, &tmK, bar, 64, y);
@@ -371,7 +411,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 }
                 for (int e = lane; e < kStageTok * 32 && ok; e += 32) {
                     const int rr = e >> 5, part = (e >> 4) & 1, ch = e & 15;  // row, K or V, 16-byte chunk
-                    if (rr < vf && pgs[rr >> 6] >= 0) continue;
+                    if ((rr & 63) < vh[rr >> 6] && pgs[rr >> 6] >= 0) continue;
                     *reinterpret_cast<uint4*>(base + (2 * part + (ch >> 3)) * kRtHalf + rr * 128 + ((ch & 7) << 4)) =
                         make_uint4(0u, 0u, 0u, 0u);
                 }
@@ -384,7 +424,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // the Quest descriptors of the blocks the window touched that lie in this share, recomputed
         // from all of each block's valid keys in global memory (the window's rows were written above
         // by this warp; at most three blocks per head)
-        if (appends && c.desc && rg == 0 && alive) {
+        if (!kSparse && appends && c.desc && rg == 0 && alive) {
             __syncwarp();
             for (int j = max(tb0, i0); j < min(N, i1); ++j) {
                 const int pg = (int)page_of(c, s, j, nullptr);
@@ -496,9 +536,11 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         float m_used = -INFINITY, l = 0.f;
         // (a wait that runs out turns this warp dead; a dead warp still takes every named barrier of the
         // loop, so the row's other warps never wait on it forever, and arrives on nothing)
+        const int hh = (kCols * cq) >> 6, hoff = (kCols * cq) & 63;  // this group's half and offset in it
         for (int q = 0; q < nproc; ++q) {
-            const int vf = stage_valid(q);
-            const int base = t_begin + kStageTok * q + kCols * cq;  // position of this group's first token
+            int jh = 0, bh = 0;
+            const int vhalf = stage_half(q, hh, jh, bh);
+            const int base = bh + hoff;  // position of this group's first token
             bool ok = alive;
             if (ok) {
                 if (lane == 0) ok = mbar_wait_sleep(&s_full[q & 1], (q >> 1) & 1, c.status);
@@ -509,7 +551,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
             if (ok) {
                 tc_fence_after();
                 tmem_ld_n<kCols>(lane_base + kColS + 128 * (q & 1) + kCols * cq, sv);
-                const int nval = min(kCols, min(vf - kCols * cq, lim - base));  // valid columns of this group
+                const int nval = min(kCols, min(vhalf - hoff, lim - base));  // valid columns of this group
                 if (nval < kCols) {
 #pragma unroll
                     for (int t = 0; t < kCols; ++t) sv[t] = t < nval ? sv[t] : -INFINITY;
@@ -636,14 +678,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     }
 }
 
-template <int kBlk>
+template <int kBlk, bool kSparse>
 int launch_rect_t(const sba_cache& c, const RtArgs& a, int row_groups, cudaStream_t stream) {
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)c.num_pages * c.H_kv * kBlk;
     if (!make_kv_tmap(&tk, c.k, rows, 64) || !make_kv_tmap(&tv, c.v, rows, 64)) return SBA_ERR_CUDA;
-    if (allow_smem<rect_tc_kernel<kBlk>>(kRtSmem) != SBA_OK) return SBA_ERR_CUDA;
+    if (allow_smem<rect_tc_kernel<kBlk, kSparse>>(kRtSmem) != SBA_OK) return SBA_ERR_CUDA;
     dim3 grid(a.num_splits, c.H_kv * row_groups, c.B);
-    return launch(rect_tc_kernel<kBlk>, grid, dim3(kRtThreads), kRtSmem, stream, tk, tv, a);
+    return launch(rect_tc_kernel<kBlk, kSparse>, grid, dim3(kRtThreads), kRtSmem, stream, tk, tv, a);
 }
 
 }  // namespace
@@ -661,7 +703,27 @@ int launch_rectify_tc(const sba_cache& c, const void* q, int f, const void* k_ne
     a.o_part = o_part;
     a.lse_part = lse_part;
     const int row_groups = (f * (c.H_q / c.H_kv) + kRtRows - 1) / kRtRows;
-    return c.b == 64 ? launch_rect_t<64>(c, a, row_groups, stream) : launch_rect_t<128>(c, a, row_groups, stream);
+    return c.b == 64 ? launch_rect_t<64, false>(c, a, row_groups, stream)
+                     : launch_rect_t<128, false>(c, a, row_groups, stream);
+}
+
+int launch_multi_query_tc(const sba_cache& c, const void* q, int M, const int32_t* sel_idx, const int32_t* sel_cnt,
+                          int n_max, float scale, int num_splits, float* o_part, float* lse_part,
+                          cudaStream_t stream) {
+    RtArgs a{};
+    a.c = c;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.M = M;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.n_max = n_max;
+    a.scale_log2 = scale * kLog2e;
+    a.num_splits = num_splits;
+    a.o_part = o_part;
+    a.lse_part = lse_part;
+    const int row_groups = (M * (c.H_q / c.H_kv) + kRtRows - 1) / kRtRows;
+    return c.b == 64 ? launch_rect_t<64, true>(c, a, row_groups, stream)
+                     : launch_rect_t<128, true>(c, a, row_groups, stream);
 }
 
 }  // namespace sba

@@ -302,7 +302,10 @@ int sba_score_select_multi(const sba_cache *c, const void *q, int32_t M, const s
  * (-inf for a row that saw no token), so sba_combine with H_q' = M*H_q merges
  * the splits into [B][M][H_q][d].  The M*G rows of a group run in row groups
  * of 128 (sba_multi_row_groups), each a CTA per split: choose num_splits so
- * that B*H_kv*row_groups*num_splits fills the GPU. */
+ * that B*H_kv*row_groups*num_splits fills the GPU.  From M*G >= 64 rows the
+ * call runs on the tcgen05 tensor cores (the rectification pipeline walking the
+ * selection), below that on mma.sync; both give the same results within the
+ * output tolerance. */
 int sba_sparse_decode_multi(const sba_cache *c, const void *q, int32_t M, const int32_t *sel_idx,
                             const int32_t *sel_cnt, int32_t n_max, float softmax_scale,
                             int32_t num_splits, float *o_part, float *lse_part, void *stream);
