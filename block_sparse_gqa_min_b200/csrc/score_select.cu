@@ -300,11 +300,25 @@ __global__ void __launch_bounds__(kThreads) score_select_kernel(ScoreArgs a) {
             if (lane == 0) lse_s[g] = M > -INFINITY ? M + logf(Z) : -INFINITY;
         }
         __syncthreads();
-        for (int j = tid; j < NC; j += kThreads) {
-            float sc = 0.f;
-            for (int g = 0; g < G; ++g)
-                sc += gate_of(__ldcg(a.scores + ((int64_t)s * c.H_q + h * G + g) * mb + j), lse_s[g], act);
-            keys[j] = orderable_key(sc);
+        // four blocks per thread and round, their G scores' loads in flight together
+        const float* sc0 = a.scores + ((int64_t)s * c.H_q + h * G) * mb;
+        for (int j0r = 0; j0r < NC; j0r += 4 * kThreads) {
+            float u[4][kMaxGroup];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int j = j0r + x * kThreads + tid;
+#pragma unroll
+                for (int g = 0; g < kMaxGroup; ++g) u[x][g] = (g < G && j < NC) ? __ldcg(sc0 + (int64_t)g * mb + j) : 0.f;
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int j = j0r + x * kThreads + tid;
+                float sc = 0.f;
+#pragma unroll
+                for (int g = 0; g < kMaxGroup; ++g)
+                    if (g < G) sc += gate_of(u[x][g], lse_s[g], act);
+                if (j < NC) keys[j] = orderable_key(sc);
+            }
         }
     }
     __syncthreads();
