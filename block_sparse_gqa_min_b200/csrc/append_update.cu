@@ -117,21 +117,39 @@ __global__ void __launch_bounds__(128) update_desc_kernel(sba_cache c, const int
         pooled[kHeadDim + tid] = lo;
         pooled[2 * kHeadDim + tid] = sum / (float)cnt;
         __syncthreads();
-        // k' = Wk . pooled : one warp per output row, lanes split the 3d inputs.
+        // k' = Wk . pooled : a warp takes four output rows at a time (their 3d inputs split over
+        // the lanes, 48 loads in flight per lane), so the rows do not wait on each other
         const int warp = tid >> 5, lane = tid & 31;
-        for (int r = warp; r < gate.dg; r += 4) {
-            const float* wr = gate.Wk + (int64_t)r * 3 * kHeadDim;
-            float acc = 0.f;
-#pragma unroll 4
-            for (int i = lane; i < 3 * kHeadDim; i += 32) acc = fmaf(__ldg(wr + i), pooled[i], acc);
+        for (int r0 = 4 * warp; r0 < gate.dg; r0 += 16) {
+            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) kproj[r] = acc;
+            for (int m = 0; m < 3 * kHeadDim / 32; ++m) {
+                const int i = lane + 32 * m;
+                const float pv = pooled[i];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    if (r0 + x < gate.dg) acc4[x] = fmaf(__ldg(gate.Wk + (int64_t)(r0 + x) * 3 * kHeadDim + i), pv, acc4[x]);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                float acc = acc4[x];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (lane == 0 && r0 + x < gate.dg) kproj[r0 + x] = acc;
+            }
         }
         __syncthreads();
-        // kg = Wq^T k' / sqrt(dg): thread t reads column t of Wq (coalesced rows).
-        float acc = 0.f;
-        for (int r = 0; r < gate.dg; ++r) acc = fmaf(__ldg(gate.Wq + (int64_t)r * kHeadDim + tid), kproj[r], acc);
+        // kg = Wq^T k' / sqrt(dg): thread t reads column t of Wq (coalesced rows), four partial sums
+        // with sixteen rows' loads in flight
+        float accp[4] = {0.f, 0.f, 0.f, 0.f};
+        int r = 0;
+        for (; r + 16 <= gate.dg; r += 16) {
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+                accp[x & 3] = fmaf(__ldg(gate.Wq + (int64_t)(r + x) * kHeadDim + tid), kproj[r + x], accp[x & 3]);
+        }
+        for (; r < gate.dg; ++r) accp[0] = fmaf(__ldg(gate.Wq + (int64_t)r * kHeadDim + tid), kproj[r], accp[0]);
+        const float acc = (accp[0] + accp[1]) + (accp[2] + accp[3]);
         c.kg[(page * c.H_kv + h) * kHeadDim + tid] = acc * rsqrtf((float)gate.dg);
     }
 }

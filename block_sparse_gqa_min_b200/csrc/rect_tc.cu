@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                 // previous stage): zero them before the tensor cores read the stage
                 bool ok = true;
                 if (nload > 0) {
-                    if (lane == 0) ok = mbar_wait(&zbar, zpar, c.status);
+                    if (lane == 0) ok = mbar_wait_sleep(&zbar, zpar, c.status);
                     zpar ^= 1u;
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                 }
@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         // wait that ran out)
         if (lane == 0 && issued) {
             umma_commit(&fin);
-            mbar_wait(&fin, 0, c.status);
+            mbar_wait_sleep(&fin, 0, c.status);
         }
         __syncwarp();
     } else {
@@ -646,7 +646,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         bool have = false;
         if (alive && nproc > 0) {
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(&pv_done[(nproc - 1) & 1], ((nproc - 1) >> 1) & 1, c.status);
+            if (lane == 0) ok = mbar_wait_sleep(&pv_done[(nproc - 1) & 1], ((nproc - 1) >> 1) & 1, c.status);
             have = __shfl_sync(0xffffffffu, ok, 0);
             if (have) tc_fence_after();
         }
