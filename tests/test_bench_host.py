@@ -62,3 +62,20 @@ def test_recorded_traffic_follows_the_source_hash(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda kernel: "0" * 64)
     assert bench.recorded_traffic("decode_step", w) is None          # kernel changed since the capture
     assert bench.recorded_traffic("decode_step", "no_such_workload") is None
+
+
+def test_rectification_counts_closed_form():
+    """R1-7B, f = 32, one sequence of 262144 tokens, 4 KV heads of G = 7 query heads:
+    bytes = every K and V row read once + the window's rows written + the touched blocks'
+    descriptors written; algorithmic flops = 4 d G sum_i (L - f + i + 1) per head (Q K^T and
+    P V over the tokens each query row sees); executed = 2 rows-tiles of 128 rows x every
+    64-token tile x 128 channels x 2 flops x 3 (S once, P V for P's hi and lo parts)."""
+    w = W.WORKLOADS["r1_7b_256k"]
+    L, f, d, G, H = 262144, 32, 128, 7, 4
+    assert bench.rect_bytes(w, [L]) == L * H * d * 2 * 2 + f * H * d * 2 * 2 + 1 * H * 512
+    alg, ex = bench.rect_flops(w, [L])
+    seen = f * (L - f) + f * (f + 1) // 2
+    assert alg == 4 * d * G * seen * H
+    assert ex == 2 * d * 128 * 2 * L * 3 * H     # 224 rows -> two 128-row tiles; L is a multiple of 64
+    # a window crossing a block boundary touches two blocks
+    assert bench.rect_bytes(w, [L + 16]) - bench.rect_bytes(w, [L]) == 16 * H * d * 2 * 2 + H * 512
