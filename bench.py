@@ -142,13 +142,39 @@ KERNEL_SOURCES = {
 }
 
 
+def strip_comments(src: str) -> str:
+    """C/C++/CUDA source without its comments and blank lines (string and character
+    literals kept as they are), so that a comment edit does not count as a kernel change."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        ch = src[i]
+        if ch in "\"'":
+            j = i + 1
+            while j < n and src[j] != ch:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(ch)
+            i += 1
+    return "\n".join(line.rstrip() for line in "".join(out).splitlines() if line.strip())
+
+
 def kernel_source_hash(kernel: str) -> str:
+    """Hash of the kernel's sources with comments removed (a recorded ncu traffic figure is
+    tied to the code it was measured on)."""
     import hashlib
 
     h = hashlib.sha256()
     for f in KERNEL_SOURCES.get(kernel, []):
-        with open(os.path.join(ROOT, "block_sparse_gqa_min_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "block_sparse_gqa_min_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()
 
 
@@ -165,7 +191,7 @@ def recorded_traffic(kernel: str, workload: str):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             fields[k.strip()] = v.strip().strip("`")
-    if fields.get("source_sha256") != kernel_source_hash(kernel):
+    if fields.get("source_sha256", "")[:64] != kernel_source_hash(kernel):
         return None
     try:
         return int(float(fields["dram_bytes_per_launch"]))

@@ -11,12 +11,13 @@
 //    contiguous cache's descriptors arrive 64 per stage in one 4-D TMA load,
 //    a paged cache's are streamed by every warp with 16-byte loads straight
 //    into registers; K/V tiles come with 2-D TMA loads (128-B swizzle);
-//  - the selection is distributed: each CTA pushes the maxima of groups of its
-//    scores to its peers (distributed shared memory); every CTA derives the same
-//    lower bound T0 of the n-th score from them (k group maxima are k distinct
-//    candidates), pushes its candidates >= T0 (score, index, page) into a
-//    cluster-wide list, and ranks that short list exactly.  Scores never reach
-//    global memory;
+//  - the selection is replicated: every CTA pushes each key (an order-preserving
+//    u32 of the block's score) to every peer as it is produced, and the maxima
+//    of groups of its keys (distributed shared memory); after one cluster
+//    barrier each CTA derives the same lower bound T0 of the n-th score from the
+//    group maxima (k group maxima are k distinct candidates), gathers the keys
+//    >= T0 from its own copy and ranks that short list exactly.  Scores never
+//    reach global memory;
 //  - partial (O, LSE) of the CTAs are pushed to the merging CTA of each output
 //    element; all pushes precede a cluster barrier, after which every CTA reads
 //    only its own shared memory;

@@ -79,3 +79,10 @@ def test_rectification_counts_closed_form():
     assert ex == 2 * d * 128 * 2 * L * 3 * H     # 224 rows -> two 128-row tiles; L is a multiple of 64
     # a window crossing a block boundary touches two blocks
     assert bench.rect_bytes(w, [L + 16]) - bench.rect_bytes(w, [L]) == 16 * H * d * 2 * 2 + H * 512
+
+
+def test_source_hash_ignores_comments_only():
+    src = 'int a = 1; // one\n/* two */ asm("x; // kept");\n'
+    assert bench.strip_comments(src) == bench.strip_comments('int a = 1;\n asm("x; // kept");  // other\n')
+    assert bench.strip_comments(src) != bench.strip_comments('int a = 2; // one\n asm("x; // kept");\n')
+    assert "// kept" in bench.strip_comments(src)  # string literals are code
